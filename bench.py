@@ -1,0 +1,368 @@
+"""Benchmark of MLA decode over a paged KV cache on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl native|reference]
+
+One step = one pass of the whole decode path over one batch: the split-KV
+scheduler kernel, the attention kernel and the split-combine kernel, with all
+inputs resident in HBM.  The default workload is the memory-bound
+configuration (batch 128, s_q 1, h_q 16, 4096 cached tokens each, 64-token
+pages, shuffled block table); its 604 MB of KV is larger than the 126 MB L2,
+so no flush is needed between steps.  Smaller workloads (--config 5) flush L2
+with a 256 MB write before every step, outside the timed events.
+
+With N > 1 (torchrun, one process per GPU) every rank decodes its own batch
+(batch-sharded replicas: sequences are independent, there is no exchange);
+`value` is the KV bytes of all ranks over the slowest rank's time.
+
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same
+workload (the project has no other reference implementation).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode TFLOPS & KV GB/s at 1 B200, as fraction of roofline, per config"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+# DRAM traffic of one attention-kernel launch on the default workload, from
+# the ncu capture summarised in profiles/ (None until captured for the
+# current kernel).
+ATTN_TRAFFIC_BYTES = None
+
+
+def _env_int(k, d):
+    try:
+        return int(os.environ.get(k, d))
+    except ValueError:
+        return d
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, uuid=None):
+        self.index = index
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = None
+            if uuid:
+                try:
+                    self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+                except Exception:
+                    self.h = None
+            if self.h is None:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+def _blas_threads() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max([x.get("num_threads", 1) for x in info] or [1])
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def _sub_work(w, batches):
+    """Algorithmic FLOPs and KV bytes of the listed sequences of workload w."""
+    from mla_decode_attention_get_b200 import inputs as I
+    sub = I.Workload(**{**w.__dict__})
+    sub.cache_seqlens = w.cache_seqlens[batches]
+    if w.indices is not None:
+        sub.indices = w.indices[batches]
+    sub.batch = len(batches)
+    return I.flops_and_bytes(sub)
+
+
+def cpu_oracle_sample(w, budget_s: float):
+    """Time the oracle, as it stands, on whole sequences of the workload until
+    `budget_s` seconds of CPU work; returns (KV GB/s, TFLOP/s, description, cores)."""
+    from oracle import mla_oracle as O
+    done, t0 = [], time.perf_counter()
+    while time.perf_counter() - t0 < budget_s and len(done) < w.batch:
+        done.append(len(done))
+        O.decode(w.q_bits, w.block_table, w.cache_seqlens, kv_bits=w.kv_bits, kv_fp8=w.kv_fp8,
+                 indices=w.indices, causal=w.causal, softmax_scale=w.softmax_scale, batches=[done[-1]])
+    el = time.perf_counter() - t0
+    flops, kv_bytes = _sub_work(w, done)
+    desc = f"{len(done)} of {w.batch} sequences of the workload, {el:.1f} s wall, numpy fp64"
+    return kv_bytes / el / 1e9, flops / el / 1e12, desc, _blas_threads()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    world = _env_int("WORLD_SIZE", 1)
+    rank = _env_int("RANK", 0)
+    local_rank = _env_int("LOCAL_RANK", 0)
+
+    from mla_decode_attention_get_b200 import inputs as I
+    hbm, tc, tc_sus, peak_src = load_peaks()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        from oracle import mla_oracle as O
+        w = I.make_config(args.config)
+        cores = _blas_threads()
+        done, elapsed = [], 0.0
+        for k in range(args.warmup + args.steps):
+            b = k % w.batch
+            t0 = time.perf_counter()
+            O.decode(w.q_bits, w.block_table, w.cache_seqlens, kv_bits=w.kv_bits, kv_fp8=w.kv_fp8,
+                     indices=w.indices, causal=w.causal, softmax_scale=w.softmax_scale, batches=[b])
+            if k >= args.warmup:
+                elapsed += time.perf_counter() - t0
+                done.append(b)
+        flops, kv_bytes = _sub_work(w, done)
+        gbs, tfl = kv_bytes / elapsed / 1e9, flops / elapsed / 1e12
+        desc = (f"each step = the oracle on one whole sequence of the workload ({args.steps} timed steps, "
+                f"{elapsed:.1f} s), numpy fp64")
+        line = {
+            "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * elapsed / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": I.CONFIG_NAMES[args.config], "config": args.config},
+            "tflops": round(tfl, 6),
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    import mla_decode_attention_get_b200 as M
+
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+
+    w = I.make_config(args.config)
+    flops, kv_bytes = I.flops_and_bytes(w)
+    t = I.to_device(w, dev)
+
+    stream = torch.cuda.current_stream(dev)
+    parts, _ = M.mla_metadata_shape(w.batch, w.s_q, w.h_q, 1, w.topk if w.fp8 else 0)
+    md = torch.empty((parts, 8), dtype=torch.int32, device=dev)
+    ns = torch.empty((w.batch * (w.s_q if w.fp8 else 1) + 1,), dtype=torch.int32, device=dev)
+    meta = lambda: M.mla_get_metadata(t["sl"], w.batch, w.s_q, w.h_q, 1, w.topk if w.fp8 else 0, md, ns)  # noqa: E731
+    meta()
+    call = M.prepare_decode(t["q"], t["kv"], t["bt"], t["sl"], 512, md, ns, w.softmax_scale, w.causal, w.fp8,
+                            t["idx"])
+    l2_small = kv_bytes < 256 * 2 ** 20
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev) if l2_small else None
+
+    def step(ev=None):
+        meta()
+        if ev is not None:
+            ev[0].record(stream)
+        call.attention()
+        if ev is not None:
+            ev[1].record(stream)
+        call.combine()
+
+    for _ in range(args.warmup):
+        if flush is not None:
+            flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if int(call._keep[9].item()) != 0:
+        raise RuntimeError(f"device error word {int(call._keep[9].item())}")
+
+    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
+    sampler = ClockSampler(dev.index if dev.index is not None else 0, uuid)
+    with sampler:
+        whole0 = torch.cuda.Event(enable_timing=True)
+        whole1 = torch.cuda.Event(enable_timing=True)
+        whole0.record(stream)
+        for k in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            step_ev[k][0].record(stream)
+            step(attn_ev[k])
+            step_ev[k][1].record(stream)
+        whole1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    if flush is None:
+        ms_total = whole0.elapsed_time(whole1)
+    else:
+        ms_total = sum(a.elapsed_time(b) for a, b in step_ev)
+    attn_ms = sum(a.elapsed_time(b) for a, b in attn_ev) / args.steps
+    if world > 1:
+        import torch.distributed as dist
+        x = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(x, op=dist.ReduceOp.MAX)
+        ms_total = float(x.item())
+    ms_step = ms_total / args.steps
+    value = kv_bytes * world / (ms_step * 1e-3) / 1e9
+    tflops = flops * world / (ms_step * 1e-3) / 1e12
+
+    # ---- end to end through the public API, host buffers, copies in the region
+    q_host = t["q"].cpu().pin_memory()
+    bt_host = t["bt"].cpu().pin_memory()
+    sl_host = t["sl"].cpu().pin_memory()
+    idx_host = t["idx"].cpu().pin_memory() if t["idx"] is not None else None
+    out_host = torch.empty((w.batch, w.s_q, w.h_q, 512), dtype=torch.bfloat16).pin_memory()
+    lse_host = torch.empty((w.batch, w.h_q, w.s_q), dtype=torch.float32).pin_memory()
+    q_dev, bt_dev, sl_dev = torch.empty_like(t["q"]), torch.empty_like(t["bt"]), torch.empty_like(t["sl"])
+    idx_dev = torch.empty_like(t["idx"]) if t["idx"] is not None else None
+    h2d = q_host.numel() * 2 + bt_host.numel() * 4 + sl_host.numel() * 4 + (idx_host.numel() * 4 if idx_host is not None else 0)
+    d2h = out_host.numel() * 2 + lse_host.numel() * 4
+
+    def e2e_step():
+        q_dev.copy_(q_host, non_blocking=True)
+        bt_dev.copy_(bt_host, non_blocking=True)
+        sl_dev.copy_(sl_host, non_blocking=True)
+        if idx_dev is not None:
+            idx_dev.copy_(idx_host, non_blocking=True)
+        md_, ns_ = M.get_mla_metadata(sl_dev, w.s_q * w.h_q, 1, s_q=w.s_q, topk=w.topk if w.fp8 else None)
+        o, l = M.flash_mla_with_kvcache(q_dev, t["kv"], bt_dev, sl_dev, 512, md_, ns_, w.softmax_scale, w.causal,
+                                        w.fp8, idx_dev)
+        out_host.copy_(o, non_blocking=True)
+        lse_host.copy_(l, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 200))
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_ms = []
+    for _ in range(e2e_steps):
+        if flush is not None:
+            flush.zero_()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        b.synchronize()
+        e_ms.append(a.elapsed_time(b))
+    e2e_value = kv_bytes * world / (statistics.mean(e_ms) * 1e-3) / 1e9
+
+    if rank != 0:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return 0
+
+    achieved = kv_bytes / (attn_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": I.CONFIG_NAMES[args.config], "config": args.config, "batch": w.batch,
+                   "s_q": w.s_q, "h_q": w.h_q, "seq_len": int(w.cache_seqlens.max()),
+                   "page": 64, "topk": w.topk, "kv_bytes": kv_bytes, "flops": flops,
+                   "l2": ("flushed before every step (256 MB write)" if flush is not None
+                          else f"inputs larger than L2 ({kv_bytes / 1e6:.0f} MB KV)"),
+                   "parallelism": f"batch-sharded replicas x{world}"},
+        "tflops": round(tflops, 3),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4), "traffic": ATTN_TRAFFIC_BYTES,
+                     "peak_source": peak_src, "kernel": "mla_decode_kernel",
+                     "kernel_ms": round(attn_ms, 5),
+                     "tensor_frac": round(flops / (attn_ms * 1e-3) / 1e12 / tc, 4)},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * args.steps,
+        "clocks": sampler.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        gbs, tfl, desc, cores = cpu_oracle_sample(w, args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                "sample": desc}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,58 @@
+// Internal interface between the C-ABI layer (mla_api.cu) and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace mla {
+
+constexpr int kPage = 64;
+constexpr int kDqk = 576;
+constexpr int kDv = 512;
+constexpr int kChunks = kDqk / 64;      // 64-dim (128-byte) column blocks of a cache row
+constexpr int kFp8Row = 656;
+constexpr int kMdWords = 8;
+constexpr int kFixedSplitCost = 5;
+
+// Row tile of the decode kernel: the number of (token, head) query rows a CTA
+// handles, chosen from the rows of one work unit.
+__host__ __device__ constexpr int tile_rows_for(int rows_per_unit) {
+  return rows_per_unit <= 16 ? 16 : (rows_per_unit <= 32 ? 32 : 64);
+}
+
+struct DecodeParams {
+  const uint8_t* kv;          // cache base (bytes)
+  int64_t kv_block_stride;    // bytes between pages
+  int num_blocks;
+  const int* block_table;
+  int bt_stride;
+  int bt_width;
+  const int* seqlens;
+  const int* indices;         // sparse path, else nullptr
+  int topk;
+  const int* tile_md;
+  const int* num_splits;
+  int num_parts;
+  int num_units;
+  uint16_t* out;              // bf16 bits
+  float* lse;
+  float* ws_o;                // [splits, rows_per_unit, 512]
+  float* ws_lse;              // [splits, rows_per_unit]
+  int* err;
+  int batch, s_q, h_q;
+  int rows_per_unit;
+  float scale_log2;           // softmax_scale * log2(e)
+  int causal;
+};
+
+// Launchers (return cudaSuccess or the launch error).
+cudaError_t launch_metadata(const int* seqlens, int batch, int s_q, int topk, int num_units, int num_parts,
+                            int* tile_md, int* num_splits, int* err, cudaStream_t stream);
+
+cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_q, const CUtensorMap& tmap_kv,
+                          int tile_rows, bool fp8, int row_tiles, cudaStream_t stream);
+
+cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream);
+
+}  // namespace mla

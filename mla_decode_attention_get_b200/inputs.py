@@ -27,7 +27,6 @@ Workload recipes follow the five decode configurations of the project
 from __future__ import annotations
 
 import dataclasses
-import math
 from typing import List, Optional
 
 import numpy as np
@@ -255,3 +254,18 @@ def flops_and_bytes(w: Workload):
                 pairs += vis * w.h_q
         kv_bytes = int(w.cache_seqlens.astype(np.int64).sum()) * D_QK * 2
     return 2 * (D_QK + D_V) * pairs, kv_bytes
+
+
+def to_device(w: Workload, dev="cuda") -> dict:
+    """Copy a workload's arrays to the device as the tensors the decode API
+    takes: q / bf16 cache as bfloat16 views of the bits, the FP8 cache as
+    uint8, tables and indices as int32."""
+    t = {"q": torch.from_numpy(w.q_bits.view(np.int16)).view(torch.bfloat16).to(dev)}
+    if w.fp8:
+        t["kv"] = torch.from_numpy(w.kv_fp8).to(dev)
+    else:
+        t["kv"] = torch.from_numpy(w.kv_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    t["bt"] = torch.from_numpy(w.block_table).to(dev)
+    t["sl"] = torch.from_numpy(w.cache_seqlens).to(dev)
+    t["idx"] = torch.from_numpy(w.indices).to(dev) if w.indices is not None else None
+    return t
