@@ -10,23 +10,29 @@
 // rows (512 e4m3 + 4 fp32 scales + 64 bf16 RoPE) -- FlashMLA walkthrough
 // (sao.pub), section "二、核心功能与架构".
 //
-// Design (one CTA = one scheduler partition x one tile of N <= 64 query rows):
-//  * Keys sit on the tensor-core M dimension ("swap AB"): for each 64-token
-//    page, S^T[64 keys, N rows] = K_page[64, 576] . Q^T is one M=64
-//    tcgen05.mma chain with S^T in TMEM; then O^T[512, N] += V^T . P^T as four
-//    M=128 MMAs (V^T is read MN-major straight from the same swizzled page
-//    tile, so V costs no extra load).  O^T lives in TMEM for the whole
-//    segment: 4N columns, plus two N-column S^T buffers.
-//  * Warp 0 streams pages with TMA (3-D tensor map, 128-byte swizzle, one
-//    page = 9 boxes of 64 tokens x 64 dims) into a 2-stage ring; warp 1
-//    issues the MMAs; warps 2-5 run the online softmax (one key per TMEM
-//    lane, warp-wide max via redux.sync, exp2 with the scale folded in, P^T
-//    written as bf16 into a swizzled K-major tile) and the epilogue.  On the
-//    FP8 sparse path warps 6-9 gather the indexed rows and dequantise them
-//    into the same bf16 page layout.
-//  * The running max is only moved when a tile's max exceeds it by more than
-//    2^8; the final division by the row sum uses the same stale max, so the
-//    result is exact.
+// Design (one CTA = one scheduler partition x one tile of 64 query rows):
+//  * Every MMA has M = 64 query rows.  Per 64-token page:
+//      S[64 rows, 64 keys]  = Q[64, 576] . K_page[64, 576]^T   36 x (K = 16)
+//      O[64 rows, 512 dims] += P[64, 64] . V_page[64, 512]       2 halves x 4 x (K = 16)
+//    V is read MN-major straight from the same swizzled page tile, so V costs
+//    no extra load.  The M = 64 accumulator layout fills 16 of the 32 lanes of
+//    each TMEM quadrant: O sits in lanes 0-15 (all 512 columns); lanes 16-31
+//    hold the two S buffers (columns 0-63, 64-127) and the query tile Q
+//    (columns 128-415, two bf16 per column), which QK reads straight from TMEM
+//    as its A operand.  With Q out of shared memory the page ring has 3 stages.
+//  * Row r of the tile belongs to threads (r % 16) and (r % 16) + 16 of
+//    softmax warp r / 16: with 16-lane TMEM accesses each of the pair holds
+//    half of the row's 64 logits (and, in the epilogue, half of its O row), so
+//    the row max / sum need one shuffle and no cross-warp synchronisation.
+//  * Warp 0 streams pages with TMA (3-D tensor map, 128-byte swizzle, one page
+//    = 9 boxes of 64 tokens x 64 dims) into the ring and warms L2 a few pages
+//    (and the next query tile) ahead; warp 1 issues the MMAs; warps 2-5 write
+//    each segment's query tile into TMEM, run the online softmax and the
+//    epilogue.  On the FP8 sparse path warps 6-9 gather the indexed rows and
+//    dequantise them into the same bf16 page layout.
+//  * The running max only moves when a page's max exceeds it by more than
+//    2^8 (per row); the final division by the row sum uses the same stale
+//    max, so the result is exact.
 //  * Every wait is bounded; on timeout the CTA raises MLA_DEVERR_TIMEOUT,
 //    drains its own copies and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
@@ -37,40 +43,51 @@
 #include "ptx_sm100.cuh"
 
 namespace mla {
+
+#ifdef MLA_TRACE
+// Opt-in pipeline trace (built only with -DMLA_TRACE): clock64() stamps of the
+// hand-offs of every page in the first kTraceCtas CTAs of row tile 0.
+constexpr int kTraceCtas = 4, kTraceEvents = 16, kTracePages = 256;
+__device__ unsigned long long g_mla_trace[kTraceCtas][kTraceEvents][kTracePages];
+#define MLA_TRACE_EV(ev, idx)                                                                   \
+  do {                                                                                          \
+    if (blockIdx.x < kTraceCtas && blockIdx.y == 0 && (idx) >= 0 && (idx) < kTracePages)        \
+      g_mla_trace[blockIdx.x][ev][idx] = clock64();                                             \
+  } while (0)
+#else
+#define MLA_TRACE_EV(ev, idx) \
+  do {                        \
+  } while (0)
+#endif
+
 namespace {
 
-constexpr int kStages = 2;
+constexpr int kRows = 64;                     // query rows per CTA = M of every MMA
+constexpr int kStages = 3;
 constexpr int kPageBytes = kPage * kDqk * 2;  // 73728: 64 tokens x 576 bf16
-constexpr int kChunkBytes = kPage * 128;      // 8192: 64 tokens x 64 dims
+constexpr int kChunkBytes = kPage * 128;      // 8192: 64 rows x 64 dims (one 128-B swizzle column)
+constexpr int kPrefetchPages = 4;             // pages warmed in L2 ahead of the TMA loads
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr int kErrBlockTable = 1, kErrIndex = 2, kErrTimeout = 4, kErrSeqlen = 8, kErrInternal = 16;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemQCol = 128;           // Q tile columns 128..415 in lanes 16-31
 
 constexpr int kWarpLoad = 0, kWarpMma = 1, kWarpSoftmax0 = 2, kWarpDequant0 = 6;
 
-template <int N>
 struct Smem {
-  static constexpr int q_chunk = N * 128;                    // one 64-dim block of N query rows
-  static constexpr int q_off = 0;
-  static constexpr int kv_off = q_off + kChunks * q_chunk;   // multiple of 1024
-  static constexpr int p_off = kv_off + kStages * kPageBytes;
-  static constexpr int red_off = p_off + N * 128;
-  static constexpr int red_bytes = 2 * 4 * N * 4;
-  static constexpr int bar_off = red_off + red_bytes;
-  // kv_full[S], kv_empty[S], s_full[2], s_empty[2], q_full, q_empty, p_full, p_empty, done, sm_sync
-  static constexpr int n_bars = 2 * kStages + 4 + 6;
+  static constexpr int kv_off = 0;                               // page ring
+  static constexpr int p_off = kv_off + kStages * kPageBytes;    // P tile: [64 rows x 64 keys] bf16
+  static constexpr int bar_off = p_off + kRows * 128;
+  // kv_full[S], kv_empty[S], s_full[2], s_empty[2], q_full, p_full, p_empty, done
+  static constexpr int n_bars = 2 * kStages + 4 + 4;
   static constexpr int info_off = bar_off + n_bars * 8;
-  static constexpr int info_bytes = kStages * 16;            // per stage: int nvalid; uint16 mask[4]
-  static constexpr int misc_off = info_off + info_bytes;     // tmem base, abort flag
+  static constexpr int info_bytes = kStages * 16;                // per stage: int nvalid; uint16 mask[4]
+  static constexpr int misc_off = info_off + info_bytes;         // tmem base, abort flag
   static constexpr int total = misc_off + 16;
   static_assert(kv_off % 1024 == 0 && p_off % 1024 == 0, "tiles must stay 1024-B aligned");
   static_assert(total <= 232448, "shared memory budget");
 };
-
-template <int N>
-constexpr uint32_t tmem_cols() {
-  return (6 * N) <= 128 ? 128u : ((6 * N) <= 256 ? 256u : 512u);
-}
 
 struct StageInfo {
   int nvalid;
@@ -84,11 +101,9 @@ struct Bars {
   uint64_t* s_full;
   uint64_t* s_empty;
   uint64_t* q_full;
-  uint64_t* q_empty;
   uint64_t* p_full;
   uint64_t* p_empty;
   uint64_t* done;
-  uint64_t* sm_sync;
 };
 
 __device__ __forceinline__ int unit_tiles(const DecodeParams& p, int u) {
@@ -150,67 +165,129 @@ __device__ __forceinline__ UnitInfo unit_info(const DecodeParams& p, int u) {
   return x;
 }
 
+__device__ __forceinline__ int page_of(const DecodeParams& p, int b, int j) {
+  return j < p.bt_width ? p.block_table[static_cast<int64_t>(b) * p.bt_stride + j] : -1;
+}
+
+// Walks the pages of a partition in order: unit u, page j of [jb, je), global
+// page index t, segment index seg.
+struct Cursor {
+  int u, j, je, t, seg;
+  bool valid;
+};
+
+__device__ __forceinline__ bool segment_bounds(const DecodeParams& p, const Partition& part, int u, int& jb,
+                                               int& je) {
+  const int n = unit_tiles(p, u);
+  jb = (u == part.u0) ? part.j0 : 0;
+  je = (u == part.u1) ? min(part.j1, n) : n;
+  return jb < je;
+}
+
+__device__ __forceinline__ void cursor_seek(const DecodeParams& p, const Partition& part, Cursor& c, int u_from) {
+  for (int u = u_from; u <= part.u1 && u < p.num_units; ++u) {
+    int jb, je;
+    if (segment_bounds(p, part, u, jb, je)) {
+      c.u = u;
+      c.j = jb;
+      c.je = je;
+      c.valid = true;
+      return;
+    }
+  }
+  c.valid = false;
+}
+
+__device__ __forceinline__ Cursor cursor_begin(const DecodeParams& p, const Partition& part) {
+  Cursor c;
+  c.t = 0;
+  c.seg = 0;
+  cursor_seek(p, part, c, part.u0);
+  return c;
+}
+
+__device__ __forceinline__ void cursor_next(const DecodeParams& p, const Partition& part, Cursor& c) {
+  ++c.t;
+  if (++c.j < c.je) return;
+  ++c.seg;
+  cursor_seek(p, part, c, c.u + 1);
+}
+
+// First query row of a unit's row tile in q (element offset of row 0).
+__device__ __forceinline__ int64_t q_tile_offset(const DecodeParams& p, const UnitInfo& ui) {
+  const int row0 = (ui.token >= 0 ? ui.token * p.h_q : 0) + blockIdx.y * kRows;
+  return static_cast<int64_t>(ui.b) * p.q_batch_stride + static_cast<int64_t>(row0) * kDqk;
+}
+
+// Rows of this CTA's tile that exist in the unit (the rest is zero padding).
+__device__ __forceinline__ int tile_valid_rows(const DecodeParams& p) {
+  return min(kRows, p.rows_per_unit - static_cast<int>(blockIdx.y) * kRows);
+}
+
 // ---------------------------------------------------------------------------
-// Warp 0: TMA loads of the query tile (once per segment) and of cache pages.
-template <int N, bool FP8>
-__device__ void load_role(const DecodeParams& p, const Partition& part, const CUtensorMap* tmap_q,
-                          const CUtensorMap* tmap_kv, uint8_t* smem, Bars bars, StageInfo* info,
-                          volatile int* abort_flag) {
-  using L = Smem<N>;
+// Warp 0 (one lane): TMA loads of cache pages with L2 warmed kPrefetchPages
+// ahead, and an L2 prefetch of the next segment's query tile.
+template <bool FP8>
+__device__ __forceinline__ void load_role(const DecodeParams& p, const Partition& part, const CUtensorMap* tmap_kv,
+                                          uint8_t* smem, Bars bars, StageInfo* info, volatile int* abort_flag) {
   const uint64_t pol_kv = l2_policy_evict_first();
-  const uint64_t pol_q = l2_policy_evict_last();
-  const int row0 = blockIdx.y * N;
-  int t = 0, seg = 0;
-  int last_t[kStages] = {-1, -1};
-  int q_last = -1;  // segment index of the last query-tile load issued
+  const uint32_t q_bytes = static_cast<uint32_t>(tile_valid_rows(p)) * kDqk * 2;
+  int t = 0;
+  int last_t[kStages];
+#pragma unroll
+  for (int s = 0; s < kStages; ++s) last_t[s] = -1;
   bool ok = true;
 
-  auto load_q = [&](const UnitInfo& ui) -> bool {
-    if (!mbar_wait(bars.q_empty, (seg & 1) ^ 1, abort_flag)) return false;
-    mbar_arrive_expect_tx(bars.q_full, kChunks * L::q_chunk);
-    const int y = (ui.token >= 0 ? ui.token * p.h_q : 0) + row0;
+  // Physical pages of the next kPrefetchPages pages, read when they are
+  // warmed in L2 so that a page's TMA load never waits on the block table.
+  int ring[kPrefetchPages];
+  auto fetch_ahead = [&](int b, int j) {
+    const int phys = page_of(p, b, j);
+    ring[j % kPrefetchPages] = phys;
+    if (phys >= 0 && phys < p.num_blocks) {
 #pragma unroll 1
-    for (int c = 0; c < kChunks; ++c)
-      tma_load_3d(smem + L::q_off + c * L::q_chunk, tmap_q, bars.q_full, 64 * c, y, ui.b, pol_q);
-    q_last = seg;
-    return true;
+      for (int c = 0; c < kChunks; ++c) tma_prefetch_3d(tmap_kv, 64 * c, 0, phys);
+    }
   };
 
   for_each_segment(p, part, [&](int u, int jb, int je) -> bool {
-    const UnitInfo ui = unit_info(p, u);
-    if (FP8) {
-      if (!load_q(ui)) { ok = false; return false; }
-      ++seg;
+    // warm the query tile of the following segment
+    if (u + 1 <= part.u1 && u + 1 < p.num_units) {
+      int jb2, je2;
+      if (segment_bounds(p, part, u + 1, jb2, je2))
+        bulk_prefetch_l2(p.q + q_tile_offset(p, unit_info(p, u + 1)), q_bytes);
+    }
+    if constexpr (FP8) {
+      return true;
+    } else {
+      const UnitInfo ui = unit_info(p, u);
+      for (int j = jb; j < min(je, jb + kPrefetchPages); ++j) fetch_ahead(ui.b, j);
+      for (int j = jb; j < je; ++j) {
+        const int s = t % kStages;
+        if (!mbar_wait(&bars.kv_empty[s], ((t / kStages) & 1) ^ 1, abort_flag)) { ok = false; return false; }
+        MLA_TRACE_EV(0, t);
+        int nv = min(kPage, ui.L - kPage * j);
+        const int phys = ring[j % kPrefetchPages];
+        if (phys < 0 || phys >= p.num_blocks) {
+          atomicOr(p.err, kErrBlockTable);
+          nv = 0;
+        }
+        info[s].nvalid = nv;
+        if (nv > 0) {
+          mbar_arrive_expect_tx(&bars.kv_full[s], kPageBytes);
+          uint8_t* dst = smem + Smem::kv_off + s * kPageBytes;
+#pragma unroll 1
+          for (int c = 0; c < kChunks; ++c)
+            tma_load_3d(dst + c * kChunkBytes, tmap_kv, &bars.kv_full[s], 64 * c, 0, phys, pol_kv);
+          last_t[s] = t;
+        } else {
+          mbar_arrive(&bars.kv_full[s]);
+        }
+        if (j + kPrefetchPages < je) fetch_ahead(ui.b, j + kPrefetchPages);
+        ++t;
+      }
       return true;
     }
-    for (int j = jb; j < je; ++j) {
-      const int s = t % kStages;
-      if (!mbar_wait(&bars.kv_empty[s], ((t / kStages) & 1) ^ 1, abort_flag)) { ok = false; return false; }
-      int nv = min(kPage, ui.L - kPage * j);
-      int phys = -1;
-      if (j < p.bt_width) phys = p.block_table[static_cast<int64_t>(ui.b) * p.bt_stride + j];
-      if (j >= p.bt_width || phys < 0 || phys >= p.num_blocks) {
-        atomicOr(p.err, kErrBlockTable);
-        nv = 0;
-      }
-      info[s].nvalid = nv;
-      if (nv > 0) {
-        mbar_arrive_expect_tx(&bars.kv_full[s], kPageBytes);
-        uint8_t* dst = smem + L::kv_off + s * kPageBytes;
-#pragma unroll 1
-        for (int c = 0; c < kChunks; ++c)
-          tma_load_3d(dst + c * kChunkBytes, tmap_kv, &bars.kv_full[s], 64 * c, 0, phys, pol_kv);
-        last_t[s] = t;
-      } else {
-        mbar_arrive(&bars.kv_full[s]);
-      }
-      if (j == jb) {
-        if (!load_q(ui)) { ok = false; return false; }
-      }
-      ++t;
-    }
-    ++seg;
-    return true;
   });
 
   if (!ok) {
@@ -223,20 +300,16 @@ __device__ void load_role(const DecodeParams& p, const Partition& part, const CU
              globaltimer_ns() - t0 < kWaitTimeoutNs) {
       }
     }
-    if (q_last >= 0) {
-      while (!mbar_try_wait(bars.q_full, q_last & 1) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
-      }
-    }
   }
 }
 
 // ---------------------------------------------------------------------------
 // Warps 6-9 (FP8 sparse path): gather the rows the indices name, dequantise
 // NoPE (e4m3 x per-128 scale) and copy RoPE into the bf16 swizzled page tile.
-template <int N>
-__device__ void dequant_role(const DecodeParams& p, const Partition& part, uint8_t* smem, Bars bars,
-                             StageInfo* info, volatile int* abort_flag, int dq) {
-  using L = Smem<N>;
+// Warp dq owns keys [16 dq, 16 dq + 16) of every tile; lane l converts NoPE
+// bytes [16 l, 16 l + 16) of a row and lanes 0-7 copy its 128 RoPE bytes.
+__device__ __forceinline__ void dequant_role(const DecodeParams& p, const Partition& part, uint8_t* smem,
+                                             Bars bars, StageInfo* info, volatile int* abort_flag, int dq) {
   const int lane = threadIdx.x & 31;
   int t = 0;
   bool ok = true;
@@ -246,7 +319,7 @@ __device__ void dequant_role(const DecodeParams& p, const Partition& part, uint8
     for (int j = jb; j < je; ++j) {
       const int s = t % kStages;
       if (!mbar_wait(&bars.kv_empty[s], ((t / kStages) & 1) ^ 1, abort_flag)) { ok = false; return false; }
-      uint8_t* stage = smem + L::kv_off + s * kPageBytes;
+      uint8_t* stage = smem + Smem::kv_off + s * kPageBytes;
       uint32_t mask = 0;
 #pragma unroll 1
       for (int kb = 0; kb < 4; ++kb) {
@@ -261,8 +334,7 @@ __device__ void dequant_role(const DecodeParams& p, const Partition& part, uint8
           if (!v && pos != -1 && lane == 0) atomicOr(p.err, kErrIndex);
           int phys = -1;
           if (v) {
-            const int page = pos >> 6;
-            phys = page < p.bt_width ? p.block_table[static_cast<int64_t>(ui.b) * p.bt_stride + page] : -1;
+            phys = page_of(p, ui.b, pos >> 6);
             if (phys < 0 || phys >= p.num_blocks) {
               if (lane == 0) atomicOr(p.err, kErrBlockTable);
               v = false;
@@ -288,7 +360,6 @@ __device__ void dequant_role(const DecodeParams& p, const Partition& part, uint8
         for (int e = 0; e < 4; ++e) {
           const int k = 16 * dq + 4 * kb + e;   // token row of the tile
           const int sw = k & 7;
-          // NoPE dims [16*lane, 16*lane + 16): block c = lane / 4, 16-B chunks 2*(lane%4) and +1
           uint32_t w[4] = {nope[e].x, nope[e].y, nope[e].z, nope[e].w};
           uint32_t o[8];
 #pragma unroll
@@ -297,20 +368,15 @@ __device__ void dequant_role(const DecodeParams& p, const Partition& part, uint8
             const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] >> 16), __NV_E4M3);
             const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo));
             const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hi));
-            const __nv_bfloat162 pa = __floats2bfloat162_rn(a.x * scale[e], a.y * scale[e]);
-            const __nv_bfloat162 pb = __floats2bfloat162_rn(b.x * scale[e], b.y * scale[e]);
-            o[2 * i] = *reinterpret_cast<const uint32_t*>(&pa);
-            o[2 * i + 1] = *reinterpret_cast<const uint32_t*>(&pb);
+            o[2 * i] = pack_bf16x2(a.x * scale[e], a.y * scale[e]);
+            o[2 * i + 1] = pack_bf16x2(b.x * scale[e], b.y * scale[e]);
           }
-          const int c = lane >> 2;
-          const int ch0 = 2 * (lane & 3);
-          uint8_t* rowp = stage + c * kChunkBytes + k * 128;
-          *reinterpret_cast<uint4*>(rowp + (((ch0) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-          *reinterpret_cast<uint4*>(rowp + (((ch0 + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
-          if (lane < 8) {
-            uint8_t* rp = stage + 8 * kChunkBytes + k * 128;
-            *reinterpret_cast<uint4*>(rp + ((lane ^ sw) << 4)) = rope[e];
-          }
+          const int c = lane >> 2;           // 64-dim block of this lane's 16 NoPE dims
+          const int ch0 = 2 * (lane & 3);    // first 16-B chunk inside the 128-B row
+          const uint32_t rowa = smem_u32(stage + c * kChunkBytes + k * 128);
+          st_shared_v4(rowa + ((ch0 ^ sw) << 4), make_uint4(o[0], o[1], o[2], o[3]));
+          st_shared_v4(rowa + (((ch0 + 1) ^ sw) << 4), make_uint4(o[4], o[5], o[6], o[7]));
+          if (lane < 8) st_shared_v4(smem_u32(stage + 8 * kChunkBytes + k * 128) + ((lane ^ sw) << 4), rope[e]);
           if (valid[e]) mask |= 1u << (4 * kb + e);
         }
       }
@@ -331,79 +397,104 @@ __device__ __forceinline__ int stage_nvalid(const StageInfo& si, bool fp8) {
 }
 
 // ---------------------------------------------------------------------------
-// Warp 1 (one lane): QK^T and PV MMAs.
-template <int N, bool FP8>
-__device__ void mma_role(const DecodeParams& p, const Partition& part, uint8_t* smem, Bars bars,
-                         const StageInfo* info, uint32_t tmem_base, volatile int* abort_flag) {
-  using L = Smem<N>;
-  constexpr uint32_t idesc_qk = idesc_bf16_f32(64, N, false, false);
-  constexpr uint32_t idesc_pv = idesc_bf16_f32(128, N, true, false);
-  const uint32_t q_addr = smem_u32(smem + L::q_off);
-  const uint32_t kv_addr = smem_u32(smem + L::kv_off);
-  const uint32_t p_addr = smem_u32(smem + L::p_off);
-  const uint32_t tmem_s[2] = {tmem_base + 4 * N, tmem_base + 5 * N};
+// Warp 1 (one lane): the QK^T and PV MMAs.  Two cursors walk the pages: QK(t)
+// is issued once page t has landed and its S buffer is free; PV(t) once the
+// softmax has written P(t).  Whichever is ready goes first (PV preferred, as
+// it releases the page's stage), so a late page never holds back the PV of
+// the previous one.
+template <bool FP8>
+__device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition& part, uint8_t* smem, Bars bars,
+                                         const StageInfo* info, uint32_t tmem_base, volatile int* abort_flag) {
+  constexpr uint32_t idesc_qk = idesc_bf16_f32(kRows, kPage, false, false);   // S = Q K^T
+  constexpr uint32_t idesc_pv = idesc_bf16_f32(kRows, 256, false, true);      // O += P V (V MN-major)
+  const uint32_t tmem_q = tmem_base + (16u << 16) + kTmemQCol;   // A operand of QK (lanes 16-31)
+  const uint64_t p_desc = sdesc_sw128(smem_u32(smem + Smem::p_off), 16, 1024);
+  uint64_t k_desc[kStages], v_desc[kStages];
+#pragma unroll
+  for (int s = 0; s < kStages; ++s) {
+    const uint32_t a = smem_u32(smem + Smem::kv_off + s * kPageBytes);
+    k_desc[s] = sdesc_sw128(a, 16, 1024);
+    v_desc[s] = sdesc_sw128(a, kChunkBytes, 1024);
+  }
+  const uint32_t tmem_s0 = tmem_base + (16u << 16);    // S buffers: lanes 16-31 of each quadrant
 
-  int t = 0, seg = 0;
-  int pv_t = -1, pv_nv = 0, pv_seg = -1, pv_stage = 0, o_seg = -1;
+  Cursor qk = cursor_begin(p, part);
+  Cursor pv = qk;
+  int o_seg = -1;
+  int qk_nv[kStages];
+#pragma unroll
+  for (int s = 0; s < kStages; ++s) qk_nv[s] = 0;
   bool ok = true;
+  uint64_t t_idle = globaltimer_ns();
+  uint32_t spins = 0;
 
-  auto issue_pv = [&]() -> bool {
-    if (!mbar_wait(bars.p_full, pv_t & 1, abort_flag)) return false;
-    tc_fence_after();
-    if (pv_nv > 0) {
-      const bool acc0 = (o_seg == pv_seg);
-      const uint32_t stage = kv_addr + pv_stage * kPageBytes;
-#pragma unroll
-      for (int jb = 0; jb < 4; ++jb) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint64_t a = sdesc_sw128(stage + (2 * jb) * kChunkBytes + k * 2048, kChunkBytes, 1024);
-          const uint64_t b = sdesc_sw128(p_addr + k * 32, 16, 1024);
-          umma_bf16(tmem_base + jb * N, a, b, idesc_pv, (acc0 || k > 0) ? 1u : 0u);
-        }
-      }
-      o_seg = pv_seg;
-    }
-    umma_commit(&bars.kv_empty[pv_stage]);
-    umma_commit(bars.p_empty);
-    return true;
-  };
-
-  for_each_segment(p, part, [&](int u, int jb, int je) -> bool {
-    (void)u;
-    for (int j = jb; j < je; ++j) {
-      const int s = t % kStages;
-      const int sb = t & 1;
-      if (!mbar_wait(&bars.kv_full[s], (t / kStages) & 1, abort_flag)) { ok = false; return false; }
-      if (j == jb && !mbar_wait(bars.q_full, seg & 1, abort_flag)) { ok = false; return false; }
-      if (!mbar_wait(&bars.s_empty[sb], ((t >> 1) & 1) ^ 1, abort_flag)) { ok = false; return false; }
+  while (pv.valid) {
+    bool progressed = false;
+    // PV(pv.t): after QK(pv.t) was issued and the softmax wrote P(pv.t)
+    if (pv.t < qk.t && mbar_test_wait(bars.p_full, pv.t & 1)) {
+      MLA_TRACE_EV(3, pv.t);
       tc_fence_after();
-      const int nv = stage_nvalid(info[s], FP8);
-      if (nv > 0) {
-        const uint32_t stage = kv_addr + s * kPageBytes;
-#pragma unroll 1
-        for (int c = 0; c < kChunks; ++c) {
+      const int s = pv.t % kStages;
+      if (qk_nv[s] > 0) {
+        const bool acc0 = (o_seg == pv.seg);
+        const uint64_t vd = v_desc[s];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const uint64_t a = sdesc_sw128(stage + c * kChunkBytes + k * 32, 16, 1024);
-            const uint64_t b = sdesc_sw128(q_addr + c * L::q_chunk + k * 32, 16, 1024);
-            umma_bf16(tmem_s[sb], a, b, idesc_qk, (c | k) != 0 ? 1u : 0u);
+            umma_bf16(tmem_base + h * 256, p_desc + ((k * 32) >> 4), vd + ((4 * h * kChunkBytes + k * 2048) >> 4),
+                      idesc_pv, (acc0 || k > 0) ? 1u : 0u);
           }
         }
+        o_seg = pv.seg;
       }
-      umma_commit(&bars.s_full[sb]);
-      if (j == je - 1) umma_commit(bars.q_empty);
-      if (pv_t >= 0 && !issue_pv()) { ok = false; return false; }
-      pv_t = t;
-      pv_nv = nv;
-      pv_seg = seg;
-      pv_stage = s;
-      ++t;
+      umma_commit(&bars.kv_empty[s]);
+      umma_commit(bars.p_empty);
+      MLA_TRACE_EV(14, pv.t);
+      cursor_next(p, part, pv);
+      progressed = true;
     }
-    ++seg;
-    return true;
-  });
-  if (ok && pv_t >= 0) ok = issue_pv();
+    // QK(qk.t): page landed, query tile of its segment loaded, S buffer free
+    if (qk.valid) {
+      const int s = qk.t % kStages;
+      const int sb = qk.t & 1;
+      const bool first = (qk.j == (qk.u == part.u0 ? part.j0 : 0));
+      if (mbar_test_wait(&bars.kv_full[s], (qk.t / kStages) & 1) &&
+          (!first || mbar_test_wait(bars.q_full, qk.seg & 1)) &&
+          mbar_test_wait(&bars.s_empty[sb], ((qk.t >> 1) & 1) ^ 1)) {
+        MLA_TRACE_EV(2, qk.t);
+        tc_fence_after();
+        const int nv = stage_nvalid(info[s], FP8);
+        qk_nv[s] = nv;
+        if (nv > 0) {
+          const uint64_t kd = k_desc[s];
+          const uint32_t d = tmem_s0 + sb * kPage;
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              // K elements [64c + 16k, +16) of Q = TMEM columns [32c + 8k, +8)
+              umma_bf16_ts(d, tmem_q + 32 * c + 8 * k, kd + ((c * kChunkBytes + k * 32) >> 4), idesc_qk,
+                           (c | k) != 0 ? 1u : 0u);
+            }
+          }
+        }
+        umma_commit(&bars.s_full[sb]);
+        MLA_TRACE_EV(12, qk.t);
+        cursor_next(p, part, qk);
+        progressed = true;
+      }
+    }
+    if (progressed) {
+      spins = 0;
+      t_idle = globaltimer_ns();
+    } else if ((++spins & 255u) == 0) {
+      if (*abort_flag || globaltimer_ns() - t_idle > kWaitTimeoutNs) {
+        ok = false;
+        break;
+      }
+    }
+  }
   if (!ok) raise_abort(abort_flag, p.err);
   // Wait until every MMA this warp issued has completed.
   umma_commit(bars.done);
@@ -413,183 +504,218 @@ __device__ void mma_role(const DecodeParams& p, const Partition& part, uint8_t* 
 }
 
 // ---------------------------------------------------------------------------
+// Warps 2-5 (whole warps): the query tile of a unit into TMEM lanes 16-31 as
+// packed bf16 pairs.  Thread (r, half) writes row r's dims
+// [128 c + 64 half, +64) for c = 0..3 and RoPE dims [512 + 32 half, +32).
+__device__ __forceinline__ void write_q_tile(const DecodeParams& p, const UnitInfo& ui, uint32_t tq_lane, int r,
+                                             int half) {
+  const bool valid = r < tile_valid_rows(p);
+  const uint4* src = reinterpret_cast<const uint4*>(p.q + q_tile_offset(p, ui) + static_cast<int64_t>(r) * kDqk);
+  uint4 buf[18];
+#pragma unroll
+  for (int c = 0; c < 2; ++c)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) buf[8 * c + i] = valid ? __ldg(src + 16 * c + 8 * half + i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    uint32_t v[32];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[4 * i] = buf[8 * c + i].x; v[4 * i + 1] = buf[8 * c + i].y;
+      v[4 * i + 2] = buf[8 * c + i].z; v[4 * i + 3] = buf[8 * c + i].w;
+    }
+    tmem_st_16x32bx2_x32u(tq_lane + 64 * c, v);
+  }
+#pragma unroll
+  for (int c = 2; c < 4; ++c)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) buf[8 * (c - 2) + i] = valid ? __ldg(src + 16 * c + 8 * half + i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) buf[16 + i] = valid ? __ldg(src + 64 + 4 * half + i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int c = 2; c < 4; ++c) {
+    uint32_t v[32];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[4 * i] = buf[8 * (c - 2) + i].x; v[4 * i + 1] = buf[8 * (c - 2) + i].y;
+      v[4 * i + 2] = buf[8 * (c - 2) + i].z; v[4 * i + 3] = buf[8 * (c - 2) + i].w;
+    }
+    tmem_st_16x32bx2_x32u(tq_lane + 64 * c, v);
+  }
+  uint32_t w[16];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    w[4 * i] = buf[16 + i].x; w[4 * i + 1] = buf[16 + i].y; w[4 * i + 2] = buf[16 + i].z; w[4 * i + 3] = buf[16 + i].w;
+  }
+#pragma unroll
+  for (int i = 2; i < 4; ++i) {
+    const uint4 x = valid ? __ldg(src + 64 + 4 * half + i) : make_uint4(0, 0, 0, 0);
+    w[4 * i] = x.x; w[4 * i + 1] = x.y; w[4 * i + 2] = x.z; w[4 * i + 3] = x.w;
+  }
+  tmem_st_16x32bx2_x16(tq_lane + 256, w);
+}
+
+// ---------------------------------------------------------------------------
 // Warps 2-5: online softmax per page and the per-segment epilogue.
-template <int N, bool FP8>
-__device__ void softmax_role(const DecodeParams& p, const Partition& part, uint8_t* smem, Bars bars,
-                             const StageInfo* info, uint32_t tmem_base, volatile int* abort_flag) {
-  using L = Smem<N>;
+template <bool FP8>
+__device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partition& part, uint8_t* smem,
+                                             Bars bars, const StageInfo* info, uint32_t tmem_base,
+                                             volatile int* abort_flag) {
   const int lane = threadIdx.x & 31;
   const int q4 = (threadIdx.x >> 5) & 3;            // TMEM lane quadrant of this warp
-  const uint32_t lane_off = static_cast<uint32_t>(32 * q4) << 16;
-  const bool key_lane = lane < 16;                  // M=64 accumulators use lanes 0-15 of each quadrant
-  const int key = 16 * q4 + lane;
-  const uint32_t tmem_s[2] = {tmem_base + 4 * N, tmem_base + 5 * N};
-  float* red_base = reinterpret_cast<float*>(smem + L::red_off);
-  uint8_t* p_tile = smem + L::p_off;
-  const int row0 = blockIdx.y * N;
+  const int half = lane >> 4;                        // which half of the row's keys / dims
+  const int r = 16 * q4 + (lane & 15);               // tile row of this thread
   const int R = p.rows_per_unit;
+  const int grow = blockIdx.y * kRows + r;           // row within the unit
+  const bool row_valid = grow < R;
+  const float scale_log2 = p.scale_log2;
+  const int h_q = p.h_q, s_q = p.s_q;
+  const int tok_dense = grow / h_q;                  // dense path: the row's query token
+  const bool causal = !FP8 && p.causal != 0;
+  const uint32_t s_taddr = tmem_base + (static_cast<uint32_t>(32 * q4 + 16) << 16);
+  const uint32_t o_taddr = tmem_base + (static_cast<uint32_t>(32 * q4) << 16);
+  const uint32_t p_row = smem_u32(smem + Smem::p_off) + r * 128;
+  const int key0 = 32 * half;                        // first key (and dim offset) of this thread's half
+  const uint32_t tq_lane = tmem_base + (static_cast<uint32_t>(32 * q4 + 16) << 16) + kTmemQCol;
 
-  float m_run[N], l_run[N];
-  int t = 0, seg = 0, sync_uses = 0;
-  bool ok = true;
-
-  auto group_sync = [&]() -> bool {
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bars.sm_sync);
-    const bool r = mbar_wait(bars.sm_sync, sync_uses & 1, abort_flag);
-    ++sync_uses;
-    return r;
+  // The query tile of the unit that follows u in this partition, if any, goes
+  // into TMEM once every QK of the current segment has been consumed.
+  auto stage_next_q = [&](int u_from) {
+    for (int u = u_from; u <= part.u1 && u < p.num_units; ++u) {
+      int jb, je;
+      if (segment_bounds(p, part, u, jb, je)) {
+        write_q_tile(p, unit_info(p, u), tq_lane, r, half);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars.q_full);
+        return;
+      }
+    }
   };
+  stage_next_q(part.u0);
+
+  int t = 0;
+  bool ok = true;
 
   for_each_segment(p, part, [&](int u, int jb, int je) -> bool {
     const UnitInfo ui = unit_info(p, u);
     if (!FP8 && lane == 0 && q4 == 0 && p.seqlens[ui.b] < 0) atomicOr(p.err, kErrSeqlen);
-#pragma unroll
-    for (int c = 0; c < N; ++c) {
-      m_run[c] = -INFINITY;
-      l_run[c] = 0.f;
-    }
+    float m_run = -INFINITY, l_run = 0.f;
     bool any_pv = false;
-    // causal limit: key position must be <= L - s_q + token(row)
-    const bool causal = !FP8 && p.causal != 0;
+    const int lim = ui.L - s_q + tok_dense + 1;      // causal: keys t < lim are visible
     for (int j = jb; j < je; ++j) {
       const int s = t % kStages;
       const int sb = t & 1;
       if (!mbar_wait(&bars.kv_full[s], (t / kStages) & 1, abort_flag)) { ok = false; return false; }
       if (!mbar_wait(&bars.s_full[sb], (t >> 1) & 1, abort_flag)) { ok = false; return false; }
+      if (lane == 0 && q4 == 2) MLA_TRACE_EV(4, t);
       tc_fence_after();
       const int nv = stage_nvalid(info[s], FP8);
-      bool kvalid;
-      if (FP8) {
-        const uint32_t m16 = info[s].mask[q4];
-        kvalid = key_lane && ((m16 >> lane) & 1u);
-      } else {
-        kvalid = key_lane && key < nv;
-      }
-      const int kpos = kPage * j + key;
-      const bool causal_pg = causal && (kPage * j + kPage - 1 > ui.L - p.s_q);
-      float* red = red_base + (t & 1) * 4 * N;
-
-      auto logit = [&](float raw, int c) -> float {
-        bool v = kvalid;
-        if (causal_pg) {
-          const int tok = (row0 + c) / p.h_q;
-          v = v && (kpos <= ui.L - p.s_q + tok);
-        }
-        return v ? raw * p.scale_log2 : -INFINITY;
-      };
-
-      // pass 1: per-row maxima of this page
-      if (nv > 0) {
-#pragma unroll
-        for (int g = 0; g < N / 16; ++g) {
-          float v[16];
-          tmem_ld16(tmem_s[sb] + lane_off + 16 * g, v);
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float mx = warp_max_f32(logit(v[c], 16 * g + c));
-            if (lane == 0) red[q4 * N + 16 * g + c] = mx;
-          }
-        }
-      }
-      if (!group_sync()) { ok = false; return false; }
-
-      // new maxima; rescale only when some row's max grew by more than 2^8
-      bool need = false;
-      if (nv > 0) {
-#pragma unroll
-        for (int c = 0; c < N; ++c) {
-          const float tm = fmaxf(fmaxf(red[c], red[N + c]), fmaxf(red[2 * N + c], red[3 * N + c]));
-          need |= tm > m_run[c] + kRescaleThreshold;
-        }
-      }
-      if (t > 0 && !mbar_wait(bars.p_empty, (t - 1) & 1, abort_flag)) { ok = false; return false; }
-      tc_fence_after();
-      if (need) {
-        if (any_pv) {
-#pragma unroll 1
-          for (int jb4 = 0; jb4 < 4; ++jb4) {
-#pragma unroll
-            for (int g = 0; g < N / 16; ++g) {
-              float v[16];
-              const uint32_t addr = tmem_base + lane_off + jb4 * N + 16 * g;
-              tmem_ld16(addr, v);
-#pragma unroll
-              for (int c = 0; c < 16; ++c) {
-                const int cc = 16 * g + c;
-                const float tm = fmaxf(fmaxf(red[cc], red[N + cc]), fmaxf(red[2 * N + cc], red[3 * N + cc]));
-                const float mn = fmaxf(m_run[cc], tm);
-                v[c] *= (mn == -INFINITY) ? 1.f : fast_exp2(m_run[cc] - mn);
-              }
-              tmem_st16(addr, v);
-            }
-          }
-        }
-#pragma unroll
-        for (int c = 0; c < N; ++c) {
-          const float tm = fmaxf(fmaxf(red[c], red[N + c]), fmaxf(red[2 * N + c], red[3 * N + c]));
-          const float mn = fmaxf(m_run[c], tm);
-          l_run[c] *= (mn == -INFINITY) ? 1.f : fast_exp2(m_run[c] - mn);
-          m_run[c] = mn;
-        }
-      }
-
-      // pass 2: P = exp2(s - m) as bf16 into the K-major swizzled P^T tile
-      if (nv > 0) {
-#pragma unroll
-        for (int g = 0; g < N / 16; ++g) {
-          float v[16];
-          tmem_ld16(tmem_s[sb] + lane_off + 16 * g, v);
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int cc = 16 * g + c;
-            const float x = logit(v[c], cc);
-            const float m_safe = m_run[cc] == -INFINITY ? 0.f : m_run[cc];
-            const float pr = key_lane ? fast_exp2(x - m_safe) : 0.f;
-            const __nv_bfloat16 pb = __float2bfloat16_rn(pr);
-            l_run[cc] += pr;
-            if (key_lane) {
-              uint8_t* dst = p_tile + cc * 128 + ((((key >> 3) ^ (cc & 7)) << 4)) + (key & 7) * 2;
-              *reinterpret_cast<__nv_bfloat16*>(dst) = pb;
-            }
-          }
-        }
-      }
+      float x[32];
+      if (nv > 0) tmem_ld_16x32bx2_x32(s_taddr + sb * kPage, x);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.s_empty[sb]);
 
+      float tmax = -INFINITY;
+      if (nv > 0) {
+        uint32_t vmask;
+        if (FP8) {
+          vmask = static_cast<uint32_t>(info[s].mask[2 * half]) |
+                  (static_cast<uint32_t>(info[s].mask[2 * half + 1]) << 16);
+        } else {
+          const int nk = min(max(nv - key0, 0), 32);
+          vmask = nk >= 32 ? 0xFFFFFFFFu : ((1u << nk) - 1u);
+          if (causal && kPage * j + key0 + 31 >= lim) {
+            const int nc = min(max(lim - kPage * j - key0, 0), 32);
+            vmask &= nc >= 32 ? 0xFFFFFFFFu : ((1u << nc) - 1u);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          x[i] = ((vmask >> i) & 1u) ? x[i] * scale_log2 : -INFINITY;
+          tmax = fmaxf(tmax, x[i]);
+        }
+      }
+      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+      const bool need = tmax > m_run + kRescaleThreshold;
+      if (lane == 0 && q4 == 2) MLA_TRACE_EV(11, t);
+
+      if (t > 0 && !mbar_wait(bars.p_empty, (t - 1) & 1, abort_flag)) { ok = false; return false; }
+      if (lane == 0 && q4 == 2) MLA_TRACE_EV(6, t);
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, need)) {
+        const float m_new = need ? fmaxf(m_run, tmax) : m_run;
+        const float alpha = (m_new == m_run) ? 1.f : fast_exp2(m_run - m_new);   // m_run = -inf -> 0
+        l_run *= alpha;
+        m_run = m_new;
+        if (__any_sync(0xffffffffu, any_pv && alpha != 1.f)) {
+          if (lane == 0 && q4 == 2) MLA_TRACE_EV(9, t);
+#pragma unroll 1
+          for (int c0 = 0; c0 < kDv; c0 += 64) {
+            float v[32];
+            tmem_ld_16x32bx2_x32(o_taddr + c0, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= alpha;
+            tmem_st_16x32bx2_x32(o_taddr + c0, v);
+          }
+        }
+      }
+
+      // P = exp2(s - m) as bf16: this thread's 64-B half of row r of the
+      // K-major swizzled P tile
+      const float m_safe = m_run == -INFINITY ? 0.f : m_run;
+      uint32_t pk[16];
+      if (nv > 0) {
+        float lsum = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float a = fast_exp2(x[2 * i] - m_safe);
+          const float b = fast_exp2(x[2 * i + 1] - m_safe);
+          lsum += a + b;
+          pk[i] = pack_bf16x2(a, b);
+        }
+        l_run += lsum;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = 0u;
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int chunk = 4 * half + c;
+        st_shared_v4(p_row + ((chunk ^ (r & 7)) << 4),
+                     make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]));
+      }
+      if (lane == 0 && q4 == 2) MLA_TRACE_EV(13, t);
+
       // a partial last page may hold non-finite padding: zero its unused V rows
       if (!FP8 && nv > 0 && nv < kPage) {
-        uint8_t* stage = smem + L::kv_off + s * kPageBytes;
+        uint8_t* stage = smem + Smem::kv_off + s * kPageBytes;
         const int nrow = kPage - nv;
         const int tid = (q4 << 5) | lane;
         for (int idx = tid; idx < nrow * 8 * 8; idx += 128) {
-          const int r = nv + idx / 64;
+          const int rr = nv + idx / 64;
           const int rem = idx % 64;
           const int c = rem / 8, ch = rem % 8;
-          *reinterpret_cast<uint4*>(stage + c * kChunkBytes + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+          st_shared_v4(smem_u32(stage + c * kChunkBytes + rr * 128 + ch * 16), make_uint4(0, 0, 0, 0));
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.p_full);
+      if (lane == 0 && q4 == 2) MLA_TRACE_EV(7, t);
       if (nv > 0) any_pv = true;
 
       if (j == je - 1) {
+        stage_next_q(u + 1);
         // ------------------------------------------------ epilogue of the segment
         if (!mbar_wait(bars.p_empty, t & 1, abort_flag)) { ok = false; return false; }
         tc_fence_after();
-        float* redl = red_base + ((t + 1) & 1) * 4 * N;
-#pragma unroll
-        for (int c = 0; c < N; ++c) {
-          float x = l_run[c];
-#pragma unroll
-          for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-          if (lane == 0) redl[q4 * N + c] = x;
-        }
-        if (!group_sync()) { ok = false; return false; }
+        const float l = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
+        const bool has = any_pv && l > 0.f;
+        const float inv = has ? 1.f / l : 0.f;
+        const float lse = has ? (m_run + log2f(l)) * kLn2 : -INFINITY;
         const int nsplit = p.num_splits[u + 1] - p.num_splits[u];
         const int split_idx = (u == part.u0 && jb == part.j0) ? part.first_split : p.num_splits[u];
         bool split = nsplit > 1;
@@ -599,83 +725,67 @@ __device__ void softmax_role(const DecodeParams& p, const Partition& part, uint8
           split = false;
         }
 #pragma unroll 1
-        for (int jb4 = 0; jb4 < 4; ++jb4) {
-          const int dim = 128 * jb4 + 32 * q4 + lane;
+        for (int c0 = 0; c0 < kDv; c0 += 64) {
+          float v[32];
+          tmem_ld_16x32bx2_x32(o_taddr + c0, v);
+          if (!row_valid) continue;
+          const int d0 = c0 + key0;      // this thread's 32 dims
+          if (split) {
+            float4* dst = reinterpret_cast<float4*>(p.ws_o + (static_cast<int64_t>(split_idx) * R + grow) * kDv + d0);
 #pragma unroll
-          for (int g = 0; g < N / 16; ++g) {
-            float v[16];
-            tmem_ld16(tmem_base + lane_off + jb4 * N + 16 * g, v);
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(v[4 * i] * inv, v[4 * i + 1] * inv, v[4 * i + 2] * inv, v[4 * i + 3] * inv);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(u) * R + grow) * kDv + d0);
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const int cc = 16 * g + c;
-              const int r = row0 + cc;
-              if (r >= R) continue;
-              const float l = redl[cc] + redl[N + cc] + redl[2 * N + cc] + redl[3 * N + cc];
-              const float val = (any_pv && l > 0.f) ? v[c] / l : 0.f;
-              if (split) {
-                p.ws_o[(static_cast<int64_t>(split_idx) * R + r) * kDv + dim] = val;
-              } else {
-                const __nv_bfloat16 ob = __float2bfloat16_rn(val);
-                p.out[(static_cast<int64_t>(u) * R + r) * kDv + dim] = *reinterpret_cast<const uint16_t*>(&ob);
-              }
-            }
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pack_bf16x2(v[8 * i] * inv, v[8 * i + 1] * inv),
+                                  pack_bf16x2(v[8 * i + 2] * inv, v[8 * i + 3] * inv),
+                                  pack_bf16x2(v[8 * i + 4] * inv, v[8 * i + 5] * inv),
+                                  pack_bf16x2(v[8 * i + 6] * inv, v[8 * i + 7] * inv));
           }
         }
-        {
-          const int k = (q4 << 5) | lane;   // this thread writes the lse of tile row k
-#pragma unroll
-          for (int c = 0; c < N; ++c) {
-            if (c != k) continue;
-            const int r = row0 + c;
-            if (r >= R) continue;
-            const float l = redl[c] + redl[N + c] + redl[2 * N + c] + redl[3 * N + c];
-            const float lse = (any_pv && l > 0.f) ? (m_run[c] + log2f(l)) * kLn2 : -INFINITY;
-            if (split) {
-              p.ws_lse[static_cast<int64_t>(split_idx) * R + r] = lse;
-            } else {
-              int b, tok, h;
-              if (FP8) { b = ui.b; tok = ui.token; h = r; }
-              else { b = ui.b; tok = r / p.h_q; h = r % p.h_q; }
-              p.lse[(static_cast<int64_t>(b) * p.h_q + h) * p.s_q + tok] = lse;
-            }
+        if (row_valid && half == 0) {
+          if (split) {
+            p.ws_lse[static_cast<int64_t>(split_idx) * R + grow] = lse;
+          } else {
+            int b, tok, h;
+            if (FP8) { b = ui.b; tok = ui.token; h = grow; }
+            else { b = ui.b; tok = tok_dense; h = grow % h_q; }
+            p.lse[(static_cast<int64_t>(b) * h_q + h) * s_q + tok] = lse;
           }
         }
         tc_fence_before();
-        if (!group_sync()) { ok = false; return false; }
+        if (lane == 0 && q4 == 2) MLA_TRACE_EV(8, t);
       }
       ++t;
     }
-    ++seg;
     return true;
   });
   if (!ok) raise_abort(abort_flag, p.err);
 }
 
 // ---------------------------------------------------------------------------
-template <int N, bool FP8>
+template <bool FP8>
 __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
-    mla_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_q,
-                      const __grid_constant__ CUtensorMap tmap_kv) {
-  using L = Smem<N>;
+    mla_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_kv) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::bar_off);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Smem::bar_off);
   Bars bars;
   bars.kv_full = bar;
   bars.kv_empty = bar + kStages;
   bars.s_full = bar + 2 * kStages;
   bars.s_empty = bar + 2 * kStages + 2;
   bars.q_full = bar + 2 * kStages + 4;
-  bars.q_empty = bar + 2 * kStages + 5;
-  bars.p_full = bar + 2 * kStages + 6;
-  bars.p_empty = bar + 2 * kStages + 7;
-  bars.done = bar + 2 * kStages + 8;
-  bars.sm_sync = bar + 2 * kStages + 9;
-  StageInfo* info = reinterpret_cast<StageInfo*>(smem + L::info_off);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::misc_off);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::misc_off + 4);
+  bars.p_full = bar + 2 * kStages + 5;
+  bars.p_empty = bar + 2 * kStages + 6;
+  bars.done = bar + 2 * kStages + 7;
+  StageInfo* info = reinterpret_cast<StageInfo*>(smem + Smem::info_off);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::misc_off);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::misc_off + 4);
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -693,20 +803,15 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
       mbar_init(&bars.s_full[i], 1);
       mbar_init(&bars.s_empty[i], 4);
     }
-    mbar_init(bars.q_full, 1);
-    mbar_init(bars.q_empty, 1);
+    mbar_init(bars.q_full, 4);
     mbar_init(bars.p_full, 4);
     mbar_init(bars.p_empty, 1);
     mbar_init(bars.done, 1);
-    mbar_init(bars.sm_sync, 4);
     fence_barrier_init();
   }
-  if (warp == kWarpLoad && lane == 0 && !FP8) {
-    prefetch_tensormap(&tmap_q);
-    prefetch_tensormap(&tmap_kv);
-  }
+  if (warp == kWarpLoad && lane == 0 && !FP8) prefetch_tensormap(&tmap_kv);
   if (warp == kWarpMma) {
-    tmem_alloc(tmem_slot, tmem_cols<N>());
+    tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -714,31 +819,32 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const Partition part = load_partition(p);
+  if (threadIdx.x == 0) MLA_TRACE_EV(10, 0);
 
   if (!*abort_flag) {
     if (warp == kWarpLoad) {
-      if (lane == 0) load_role<N, FP8>(p, part, &tmap_q, &tmap_kv, smem, bars, info, abort_flag);
+      if (lane == 0) load_role<FP8>(p, part, &tmap_kv, smem, bars, info, abort_flag);
     } else if (warp == kWarpMma) {
-      if (lane == 0) mma_role<N, FP8>(p, part, smem, bars, info, tmem_base, abort_flag);
-    } else if (warp < kWarpDequant0) {
-      softmax_role<N, FP8>(p, part, smem, bars, info, tmem_base, abort_flag);
+      if (lane == 0) mma_role<FP8>(p, part, smem, bars, info, tmem_base, abort_flag);
+    } else if (warp >= kWarpSoftmax0 && warp < kWarpDequant0) {
+      softmax_role<FP8>(p, part, smem, bars, info, tmem_base, abort_flag);
     } else if (FP8) {
-      dequant_role<N>(p, part, smem, bars, info, abort_flag, warp - kWarpDequant0);
+      dequant_role(p, part, smem, bars, info, abort_flag, warp - kWarpDequant0);
     }
   }
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) MLA_TRACE_EV(10, 1);
   tc_fence_after();
   if (warp == kWarpMma) {
     __syncwarp();
-    tmem_dealloc(tmem_base, tmem_cols<N>());
+    tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
-template <int N, bool FP8>
-cudaError_t launch_one(const DecodeParams& p, const CUtensorMap& tq, const CUtensorMap& tkv, int row_tiles,
-                       cudaStream_t stream) {
-  constexpr int smem = Smem<N>::total;
+template <bool FP8>
+cudaError_t launch_one(const DecodeParams& p, const CUtensorMap& tkv, int row_tiles, cudaStream_t stream) {
+  constexpr int smem = Smem::total;
   // The shared-memory opt-in is per device; remember which devices have it.
   static unsigned long long configured = 0;
   int dev = 0;
@@ -746,28 +852,32 @@ cudaError_t launch_one(const DecodeParams& p, const CUtensorMap& tq, const CUten
   if (e != cudaSuccess) return e;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(__atomic_load_n(&configured, __ATOMIC_ACQUIRE) & bit)) {
-    e = cudaFuncSetAttribute(mla_decode_kernel<N, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(mla_decode_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     __atomic_fetch_or(&configured, bit, __ATOMIC_RELEASE);
   }
   dim3 grid(p.num_parts, row_tiles);
-  mla_decode_kernel<N, FP8><<<grid, FP8 ? 320 : 192, smem, stream>>>(p, tq, tkv);
+  mla_decode_kernel<FP8><<<grid, FP8 ? 320 : 192, smem, stream>>>(p, tkv);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_q, const CUtensorMap& tmap_kv,
-                          int tile_rows, bool fp8, int row_tiles, cudaStream_t stream) {
-  switch (tile_rows) {
-    case 16: return fp8 ? launch_one<16, true>(p, tmap_q, tmap_kv, row_tiles, stream)
-                        : launch_one<16, false>(p, tmap_q, tmap_kv, row_tiles, stream);
-    case 32: return fp8 ? launch_one<32, true>(p, tmap_q, tmap_kv, row_tiles, stream)
-                        : launch_one<32, false>(p, tmap_q, tmap_kv, row_tiles, stream);
-    case 64: return fp8 ? launch_one<64, true>(p, tmap_q, tmap_kv, row_tiles, stream)
-                        : launch_one<64, false>(p, tmap_q, tmap_kv, row_tiles, stream);
-    default: return cudaErrorInvalidValue;
-  }
+#ifdef MLA_TRACE
+extern "C" __attribute__((visibility("default"))) int mla_trace_copy(void* host_dst, size_t bytes) {
+  if (bytes > sizeof(g_mla_trace)) bytes = sizeof(g_mla_trace);
+  return cudaMemcpyFromSymbol(host_dst, g_mla_trace, bytes) == cudaSuccess ? 0 : 4;
+}
+extern "C" __attribute__((visibility("default"))) int mla_trace_clear() {
+  static unsigned long long zeros[kTraceCtas][kTraceEvents][kTracePages];
+  return cudaMemcpyToSymbol(g_mla_trace, zeros, sizeof(zeros)) == cudaSuccess ? 0 : 4;
+}
+#endif
+
+cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, int tile_rows, bool fp8, int row_tiles,
+                          cudaStream_t stream) {
+  if (tile_rows != kRows) return cudaErrorInvalidValue;
+  return fp8 ? launch_one<true>(p, tmap_kv, row_tiles, stream) : launch_one<false>(p, tmap_kv, row_tiles, stream);
 }
 
 }  // namespace mla

@@ -114,6 +114,8 @@ int prepare(const mla_decode_args* a, Plan* pl, mla::DecodeParams* kp) {
   if (a->workspace_bytes < workspace_need(*pl, a->num_parts)) return MLA_ERR_WORKSPACE;
 
   std::memset(kp, 0, sizeof(*kp));
+  kp->q = static_cast<const uint16_t*>(a->q);
+  kp->q_batch_stride = a->q_batch_stride;
   kp->kv = static_cast<const uint8_t*>(a->k_cache);
   kp->kv_block_stride = a->k_block_stride;
   kp->num_blocks = a->num_blocks;
@@ -191,18 +193,13 @@ int mla_decode_attention(const mla_decode_args* a, void* stream) {
   mla::DecodeParams kp;
   int st = prepare(a, &pl, &kp);
   if (st != MLA_OK) return st;
-  CUtensorMap tq, tkv;
-  std::memset(&tq, 0, sizeof(tq));
+  CUtensorMap tkv;
   std::memset(&tkv, 0, sizeof(tkv));
-  const uint64_t rows = uint64_t(a->s_q) * a->h_q;
-  if (!encode_bf16_map(&tq, a->q, rows, uint64_t(a->batch), uint64_t(kDqk) * 2, uint64_t(a->q_batch_stride) * 2,
-                       pl.tile_rows))
-    return MLA_ERR_CUDA;
   if (!a->is_fp8 && !encode_bf16_map(&tkv, a->k_cache, uint64_t(kPage), uint64_t(a->num_blocks),
                                      uint64_t(kDqk) * 2, uint64_t(a->k_block_stride), kPage))
     return MLA_ERR_CUDA;
   const cudaError_t e =
-      mla::launch_decode(kp, tq, tkv, pl.tile_rows, a->is_fp8 != 0, pl.row_tiles, static_cast<cudaStream_t>(stream));
+      mla::launch_decode(kp, tkv, pl.tile_rows, a->is_fp8 != 0, pl.row_tiles, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

@@ -16,12 +16,15 @@ constexpr int kMdWords = 8;
 constexpr int kFixedSplitCost = 5;
 
 // Row tile of the decode kernel: the number of (token, head) query rows a CTA
-// handles, chosen from the rows of one work unit.
+// handles (the M of every tensor-core MMA); units with fewer rows leave the
+// rest of the tile as zero padding.
 __host__ __device__ constexpr int tile_rows_for(int rows_per_unit) {
-  return rows_per_unit <= 16 ? 16 : (rows_per_unit <= 32 ? 32 : 64);
+  return (void)rows_per_unit, 64;
 }
 
 struct DecodeParams {
+  const uint16_t* q;          // bf16 bits [batch, s_q, h_q, 576]
+  int64_t q_batch_stride;     // elements between batch entries
   const uint8_t* kv;          // cache base (bytes)
   int64_t kv_block_stride;    // bytes between pages
   int num_blocks;
@@ -50,8 +53,8 @@ struct DecodeParams {
 cudaError_t launch_metadata(const int* seqlens, int batch, int s_q, int topk, int num_units, int num_parts,
                             int* tile_md, int* num_splits, int* err, cudaStream_t stream);
 
-cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_q, const CUtensorMap& tmap_kv,
-                          int tile_rows, bool fp8, int row_tiles, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, int tile_rows, bool fp8, int row_tiles,
+                          cudaStream_t stream);
 
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream);
 
