@@ -149,6 +149,32 @@ MLA_API int mla_decode_attention(const mla_decode_args* args, void* stream);
 /* The LSE-weighted combine of split results alone (after mla_decode_attention). */
 MLA_API int mla_decode_combine(const mla_decode_args* args, void* stream);
 
+/*
+ * Decode (same arguments and results as mla_decode) for callers that cannot
+ * allocate device memory themselves: code that is handed its buffers by a
+ * host program and may not create allocations of its own (a plugin inside a
+ * serving process whose memory is budgeted up front), or code that must stay
+ * off cudaMalloc / cudaFree because those calls can synchronise the device.
+ * The pages have no counterpart to this entry point.
+ *
+ * args->workspace and args->workspace_bytes are ignored: the split-KV
+ * partial results go to one scratch array built into the library, of
+ * MLA_NOALLOC_SCRATCH_BYTES bytes on every GPU that loads the library, held
+ * until the process exits.  A plan needing more than that (see
+ * mla_workspace_bytes) returns MLA_ERR_WORKSPACE before anything is
+ * launched.  No allocation is made by this call.
+ *  - The first call on a device looks the array's device address up with
+ *    cudaGetSymbolAddress (once per device, with that device current); make
+ *    that first call before any stream capture begins.
+ *  - All calls share the one array, and it keeps whatever the last call left
+ *    in it.  Nothing in it needs to start at zero: every slot the combine
+ *    kernel reads is written earlier in the same call.  Calls whose kernels
+ *    overlap on the GPU (different streams, no ordering between them) race
+ *    on the array and corrupt each other's results; order them.
+ */
+#define MLA_NOALLOC_SCRATCH_BYTES (64u << 20)
+MLA_API int mla_decode_noalloc(const mla_decode_args* args, void* stream);
+
 /* Human-readable name of a status code (static string). */
 MLA_API const char* mla_status_string(int status);
 

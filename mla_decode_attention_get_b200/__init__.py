@@ -26,8 +26,8 @@ from . import _abi
 from ._abi import MlaError, D_QK, D_V, PAGE_SIZE, FP8_ROW_BYTES
 
 __all__ = ["get_mla_metadata", "flash_mla_with_kvcache", "MlaError", "mla_get_metadata", "mla_decode",
-           "mla_decode_attention", "mla_decode_combine", "mla_metadata_shape", "mla_workspace_bytes",
-           "DecodeCall"]
+           "mla_decode_attention", "mla_decode_combine", "mla_decode_noalloc", "mla_metadata_shape",
+           "mla_workspace_bytes", "DecodeCall"]
 
 
 def _stream_ptr(device) -> int:
@@ -104,6 +104,11 @@ class DecodeCall:
     def decode(self, stream=None):
         self._call(_abi.lib().mla_decode, "mla_decode", stream)
 
+    def decode_noalloc(self, stream=None):
+        """The same decode through mla_decode_noalloc: the library's built-in
+        scratch array replaces this call's workspace tensor."""
+        self._call(_abi.lib().mla_decode_noalloc, "mla_decode_noalloc", stream)
+
     def attention(self, stream=None):
         self._call(_abi.lib().mla_decode_attention, "mla_decode_attention", stream)
 
@@ -113,6 +118,10 @@ class DecodeCall:
 
 def mla_decode(call: DecodeCall) -> None:
     call.decode()
+
+
+def mla_decode_noalloc(call: DecodeCall) -> None:
+    call.decode_noalloc()
 
 
 def mla_decode_attention(call: DecodeCall) -> None:
