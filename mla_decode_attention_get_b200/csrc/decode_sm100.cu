@@ -49,12 +49,27 @@ namespace mla {
 // hand-offs of every page in the first kTraceCtas CTAs of row tile 0.
 constexpr int kTraceCtas = 4, kTraceEvents = 16, kTracePages = 256;
 __device__ unsigned long long g_mla_trace[kTraceCtas][kTraceEvents][kTracePages];
+// globaltimer at the start and end of every CTA (x + 1024 * y), and its SM
+__device__ unsigned long long g_mla_trace_span[3][4096];
 #define MLA_TRACE_EV(ev, idx)                                                                   \
   do {                                                                                          \
     if (blockIdx.x < kTraceCtas && blockIdx.y == 0 && (idx) >= 0 && (idx) < kTracePages)        \
       g_mla_trace[blockIdx.x][ev][idx] = clock64();                                             \
   } while (0)
+#define MLA_TRACE_SPAN(which)                                                                   \
+  do {                                                                                          \
+    const unsigned id = blockIdx.x + 1024u * blockIdx.y;                                        \
+    if (id < 4096u) {                                                                           \
+      g_mla_trace_span[which][id] = globaltimer_ns();                                           \
+      unsigned smid;                                                                            \
+      asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));                                         \
+      g_mla_trace_span[2][id] = smid;                                                           \
+    }                                                                                           \
+  } while (0)
 #else
+#define MLA_TRACE_SPAN(which) \
+  do {                        \
+  } while (0)
 #define MLA_TRACE_EV(ev, idx) \
   do {                        \
   } while (0)
@@ -261,7 +276,16 @@ __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition
       return true;
     } else {
       const UnitInfo ui = unit_info(p, u);
-      for (int j = jb; j < min(je, jb + kPrefetchPages); ++j) fetch_ahead(ui.b, j);
+      // read the first pages' table entries together, then warm L2
+      const int jn = min(je, jb + kPrefetchPages);
+      for (int j = jb; j < jn; ++j) ring[j % kPrefetchPages] = page_of(p, ui.b, j);
+      for (int j = jb; j < jn; ++j) {
+        const int phys = ring[j % kPrefetchPages];
+        if (phys >= 0 && phys < p.num_blocks) {
+#pragma unroll 1
+          for (int c = 0; c < kChunks; ++c) tma_prefetch_3d(tmap_kv, 64 * c, 0, phys);
+        }
+      }
       for (int j = jb; j < je; ++j) {
         const int s = t % kStages;
         if (!mbar_wait(&bars.kv_empty[s], ((t / kStages) & 1) ^ 1, abort_flag)) { ok = false; return false; }
@@ -397,7 +421,9 @@ __device__ __forceinline__ int stage_nvalid(const StageInfo& si, bool fp8) {
 }
 
 // ---------------------------------------------------------------------------
-// Warp 1 (one lane): the QK^T and PV MMAs.  Two cursors walk the pages: QK(t)
+// Warp 1 (whole warp, one elected lane issues): the QK^T and PV MMAs.  Lane 0
+// tests the barriers and broadcasts, so control flow stays warp-uniform and
+// the MMA operands stay uniform.  Two cursors walk the pages: QK(t)
 // is issued once page t has landed and its S buffer is free; PV(t) once the
 // softmax has written P(t).  Whichever is ready goes first (PV preferred, as
 // it releases the page's stage), so a late page never holds back the PV of
@@ -428,11 +454,16 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
   uint64_t t_idle = globaltimer_ns();
   uint32_t spins = 0;
 
+  const int lane = threadIdx.x & 31;
+  auto ready = [&](uint64_t* bar, uint32_t parity) -> bool {
+    return __shfl_sync(0xffffffffu, lane == 0 ? (mbar_test_wait(bar, parity) ? 1 : 0) : 0, 0) != 0;
+  };
+
   while (pv.valid) {
     bool progressed = false;
     // PV(pv.t): after QK(pv.t) was issued and the softmax wrote P(pv.t)
-    if (pv.t < qk.t && mbar_test_wait(bars.p_full, pv.t & 1)) {
-      MLA_TRACE_EV(3, pv.t);
+    if (pv.t < qk.t && ready(bars.p_full, pv.t & 1)) {
+      if (lane == 0) MLA_TRACE_EV(3, pv.t);
       tc_fence_after();
       const int s = pv.t % kStages;
       if (qk_nv[s] > 0) {
@@ -442,15 +473,15 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            umma_bf16(tmem_base + h * 256, p_desc + ((k * 32) >> 4), vd + ((4 * h * kChunkBytes + k * 2048) >> 4),
-                      idesc_pv, (acc0 || k > 0) ? 1u : 0u);
+            umma_bf16_elect(tmem_base + h * 256, p_desc + ((k * 32) >> 4),
+                            vd + ((4 * h * kChunkBytes + k * 2048) >> 4), idesc_pv, (acc0 || k > 0) ? 1u : 0u);
           }
         }
         o_seg = pv.seg;
       }
-      umma_commit(&bars.kv_empty[s]);
-      umma_commit(bars.p_empty);
-      MLA_TRACE_EV(14, pv.t);
+      umma_commit_elect(&bars.kv_empty[s]);
+      umma_commit_elect(bars.p_empty);
+      if (lane == 0) MLA_TRACE_EV(14, pv.t);
       cursor_next(p, part, pv);
       progressed = true;
     }
@@ -459,10 +490,9 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
       const int s = qk.t % kStages;
       const int sb = qk.t & 1;
       const bool first = (qk.j == (qk.u == part.u0 ? part.j0 : 0));
-      if (mbar_test_wait(&bars.kv_full[s], (qk.t / kStages) & 1) &&
-          (!first || mbar_test_wait(bars.q_full, qk.seg & 1)) &&
-          mbar_test_wait(&bars.s_empty[sb], ((qk.t >> 1) & 1) ^ 1)) {
-        MLA_TRACE_EV(2, qk.t);
+      if (ready(&bars.kv_full[s], (qk.t / kStages) & 1) && (!first || ready(bars.q_full, qk.seg & 1)) &&
+          ready(&bars.s_empty[sb], ((qk.t >> 1) & 1) ^ 1)) {
+        if (lane == 0) MLA_TRACE_EV(2, qk.t);
         tc_fence_after();
         const int nv = stage_nvalid(info[s], FP8);
         qk_nv[s] = nv;
@@ -474,13 +504,13 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               // K elements [64c + 16k, +16) of Q = TMEM columns [32c + 8k, +8)
-              umma_bf16_ts(d, tmem_q + 32 * c + 8 * k, kd + ((c * kChunkBytes + k * 32) >> 4), idesc_qk,
-                           (c | k) != 0 ? 1u : 0u);
+              umma_bf16_ts_elect(d, tmem_q + 32 * c + 8 * k, kd + ((c * kChunkBytes + k * 32) >> 4), idesc_qk,
+                                 (c | k) != 0 ? 1u : 0u);
             }
           }
         }
-        umma_commit(&bars.s_full[sb]);
-        MLA_TRACE_EV(12, qk.t);
+        umma_commit_elect(&bars.s_full[sb]);
+        if (lane == 0) MLA_TRACE_EV(12, qk.t);
         cursor_next(p, part, qk);
         progressed = true;
       }
@@ -489,18 +519,20 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
       spins = 0;
       t_idle = globaltimer_ns();
     } else if ((++spins & 255u) == 0) {
-      if (*abort_flag || globaltimer_ns() - t_idle > kWaitTimeoutNs) {
+      const bool give_up = *abort_flag || globaltimer_ns() - t_idle > kWaitTimeoutNs;
+      if (__shfl_sync(0xffffffffu, give_up ? 1 : 0, 0)) {
         ok = false;
         break;
       }
     }
   }
-  if (!ok) raise_abort(abort_flag, p.err);
+  if (!ok && lane == 0) raise_abort(abort_flag, p.err);
   // Wait until every MMA this warp issued has completed.
-  umma_commit(bars.done);
+  umma_commit_elect(bars.done);
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bars.done, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
   }
+  __syncwarp();
 }
 
 // ---------------------------------------------------------------------------
@@ -820,12 +852,13 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
   const uint32_t tmem_base = *tmem_slot;
   const Partition part = load_partition(p);
   if (threadIdx.x == 0) MLA_TRACE_EV(10, 0);
+  if (threadIdx.x == 0) MLA_TRACE_SPAN(0);
 
   if (!*abort_flag) {
     if (warp == kWarpLoad) {
       if (lane == 0) load_role<FP8>(p, part, &tmap_kv, smem, bars, info, abort_flag);
     } else if (warp == kWarpMma) {
-      if (lane == 0) mma_role<FP8>(p, part, smem, bars, info, tmem_base, abort_flag);
+      mma_role<FP8>(p, part, smem, bars, info, tmem_base, abort_flag);
     } else if (warp >= kWarpSoftmax0 && warp < kWarpDequant0) {
       softmax_role<FP8>(p, part, smem, bars, info, tmem_base, abort_flag);
     } else if (FP8) {
@@ -835,6 +868,7 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) MLA_TRACE_EV(10, 1);
+  if (threadIdx.x == 0) MLA_TRACE_SPAN(1);
   tc_fence_after();
   if (warp == kWarpMma) {
     __syncwarp();
@@ -867,6 +901,10 @@ cudaError_t launch_one(const DecodeParams& p, const CUtensorMap& tkv, int row_ti
 extern "C" __attribute__((visibility("default"))) int mla_trace_copy(void* host_dst, size_t bytes) {
   if (bytes > sizeof(g_mla_trace)) bytes = sizeof(g_mla_trace);
   return cudaMemcpyFromSymbol(host_dst, g_mla_trace, bytes) == cudaSuccess ? 0 : 4;
+}
+extern "C" __attribute__((visibility("default"))) int mla_trace_span_copy(void* host_dst, size_t bytes) {
+  if (bytes > sizeof(g_mla_trace_span)) bytes = sizeof(g_mla_trace_span);
+  return cudaMemcpyFromSymbol(host_dst, g_mla_trace_span, bytes) == cudaSuccess ? 0 : 4;
 }
 extern "C" __attribute__((visibility("default"))) int mla_trace_clear() {
   static unsigned long long zeros[kTraceCtas][kTraceEvents][kTracePages];
