@@ -36,10 +36,10 @@ METRIC = "MLA decode TFLOPS & KV GB/s at 1 B200, as fraction of roofline, per co
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
-# DRAM traffic of one attention-kernel launch on the default workload, from
-# the ncu capture summarised in profiles/ (None until captured for the
-# current kernel).
-ATTN_TRAFFIC_BYTES = None
+# DRAM traffic (read + write bytes) of one attention-kernel launch on the
+# default workload, from one ncu capture of the current kernel; None when the
+# kernel changed since or for other workloads.
+ATTN_TRAFFIC_BYTES = {2: 629_760_000}
 
 
 def _env_int(k, d):
@@ -346,7 +346,7 @@ def main():
                    "parallelism": f"batch-sharded replicas x{world}"},
         "tflops": round(tflops, 3),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(achieved / hbm, 4), "traffic": ATTN_TRAFFIC_BYTES,
+                     "frac": round(achieved / hbm, 4), "traffic": ATTN_TRAFFIC_BYTES.get(args.config),
                      "peak_source": peak_src, "kernel": "mla_decode_kernel",
                      "kernel_ms": round(attn_ms, 5),
                      "tensor_frac": round(flops / (attn_ms * 1e-3) / 1e12 / tc, 4)},
