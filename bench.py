@@ -249,7 +249,9 @@ def main():
     if int(call._keep[9].item()) != 0:
         raise RuntimeError(f"device error word {int(call._keep[9].item())}")
 
-    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # Timed region: K steps between a barrier and a device synchronisation on
+    # both sides, one event pair around the whole loop (per-step pairs when
+    # L2 is flushed between steps, so that the flushes stay outside).
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     if world > 1:
         torch.distributed.barrier()
@@ -266,9 +268,10 @@ def main():
         for k in range(args.steps):
             if flush is not None:
                 flush.zero_()
-            step_ev[k][0].record(stream)
-            step(attn_ev[k])
-            step_ev[k][1].record(stream)
+                step_ev[k][0].record(stream)
+            step()
+            if flush is not None:
+                step_ev[k][1].record(stream)
         whole1.record(stream)
         torch.cuda.synchronize()
     if world > 1:
@@ -277,6 +280,16 @@ def main():
         ms_total = whole0.elapsed_time(whole1)
     else:
         ms_total = sum(a.elapsed_time(b) for a, b in step_ev)
+
+    # The attention kernel's own duration: the same K steps again, with an
+    # event pair around every attention launch.
+    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        step(attn_ev[k])
+    torch.cuda.synchronize()
     attn_ms = sum(a.elapsed_time(b) for a, b in attn_ev) / args.steps
     if world > 1:
         import torch.distributed as dist

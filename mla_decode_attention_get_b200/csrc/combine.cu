@@ -12,6 +12,7 @@
 #include <cuda_bf16.h>
 
 #include "mla_kernels.cuh"
+#include "ptx_sm100.cuh"
 
 namespace mla {
 namespace {
@@ -19,6 +20,8 @@ namespace {
 constexpr int kRowsPerCta = 4;  // one warp per row
 
 __global__ void __launch_bounds__(32 * kRowsPerCta) combine_kernel(const DecodeParams p) {
+  grid_dependency_wait();        // the attention kernel's partials and outputs
+  grid_launch_dependents();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int u = blockIdx.x;
@@ -35,8 +38,16 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) combine_kernel(const DecodeP
   uint2* orow = reinterpret_cast<uint2*>(p.out + (static_cast<int64_t>(u) * R + r) * kDv);
   float* lse_out = p.lse + (static_cast<int64_t>(b) * p.h_q + h) * p.s_q + tok;
 
+  // lane k holds the log-sum-exp of splits k, k + 32, ...
   float mx = -INFINITY;
-  for (int s = lane; s < n; s += 32) mx = fmaxf(mx, p.ws_lse[static_cast<int64_t>(s0 + s) * R + r]);
+  float l_reg[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int sidx = lane + 32 * i;
+    l_reg[i] = sidx < n ? p.ws_lse[static_cast<int64_t>(s0 + sidx) * R + r] : -INFINITY;
+    mx = fmaxf(mx, l_reg[i]);
+  }
+  for (int sidx = lane + 128; sidx < n; sidx += 32) mx = fmaxf(mx, p.ws_lse[static_cast<int64_t>(s0 + sidx) * R + r]);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
 
@@ -47,26 +58,54 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) combine_kernel(const DecodeP
     return;
   }
   float sum = 0.f;
-  for (int s = lane; s < n; s += 32) sum += expf(p.ws_lse[static_cast<int64_t>(s0 + s) * R + r] - mx);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) sum += expf(l_reg[i] - mx);
+  for (int sidx = lane + 128; sidx < n; sidx += 32) sum += expf(p.ws_lse[static_cast<int64_t>(s0 + sidx) * R + r] - mx);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
   const float lse = mx + logf(sum);
+  float w_reg[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) w_reg[i] = expf(l_reg[i] - lse);
 
   float4 acc[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < n; ++s) {
-    const int64_t row = static_cast<int64_t>(s0 + s) * R + r;
-    const float w = expf(p.ws_lse[row] - lse);
-    if (w == 0.f) continue;
-    const float4* src = reinterpret_cast<const float4*>(p.ws_o + row * kDv);
+  auto weight = [&](int sidx) -> float {
+    if (sidx < 128) {
+      float w = w_reg[0];
+#pragma unroll
+      for (int i = 1; i < 4; ++i) w = (sidx >> 5) == i ? w_reg[i] : w;
+      return __shfl_sync(0xffffffffu, w, sidx & 31);
+    }
+    return expf(p.ws_lse[static_cast<int64_t>(s0 + sidx) * R + r] - lse);
+  };
+  int sidx = 0;
+  for (; sidx + 1 < n; sidx += 2) {
+    const float wa = weight(sidx), wb = weight(sidx + 1);
+    const float4* a4 = reinterpret_cast<const float4*>(p.ws_o + (static_cast<int64_t>(s0 + sidx) * R + r) * kDv);
+    const float4* b4 = reinterpret_cast<const float4*>(p.ws_o + (static_cast<int64_t>(s0 + sidx + 1) * R + r) * kDv);
+    float4 va[4], vb[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) { va[k] = a4[lane + 32 * k]; vb[k] = b4[lane + 32 * k]; }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const float4 v = src[lane + 32 * k];
-      acc[k].x += w * v.x;
-      acc[k].y += w * v.y;
-      acc[k].z += w * v.z;
-      acc[k].w += w * v.w;
+      acc[k].x += wa * va[k].x + wb * vb[k].x;
+      acc[k].y += wa * va[k].y + wb * vb[k].y;
+      acc[k].z += wa * va[k].z + wb * vb[k].z;
+      acc[k].w += wa * va[k].w + wb * vb[k].w;
+    }
+  }
+  if (sidx < n) {
+    const float wa = weight(sidx);
+    const float4* a4 = reinterpret_cast<const float4*>(p.ws_o + (static_cast<int64_t>(s0 + sidx) * R + r) * kDv);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 v = a4[lane + 32 * k];
+      acc[k].x += wa * v.x;
+      acc[k].y += wa * v.y;
+      acc[k].z += wa * v.z;
+      acc[k].w += wa * v.w;
     }
   }
 #pragma unroll
@@ -82,8 +121,7 @@ __global__ void __launch_bounds__(32 * kRowsPerCta) combine_kernel(const DecodeP
 
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream) {
   dim3 grid(p.num_units, (p.rows_per_unit + kRowsPerCta - 1) / kRowsPerCta);
-  combine_kernel<<<grid, 32 * kRowsPerCta, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_dependent(combine_kernel, grid, dim3(32 * kRowsPerCta), 0, stream, p);
 }
 
 }  // namespace mla

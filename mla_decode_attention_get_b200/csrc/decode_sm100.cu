@@ -819,12 +819,9 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::misc_off + 4);
 
+  const bool misaligned = (smem_u32(smem) & 1023u) != 0;
   if (threadIdx.x == 0) {
-    *abort_flag = 0;
-    if ((smem_u32(smem) & 1023u) != 0) {
-      *abort_flag = 1;
-      atomicOr(p.err, kErrInternal);
-    }
+    *abort_flag = misaligned ? 1 : 0;
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars.kv_full[s], FP8 ? 4 : 1);
       mbar_init(&bars.kv_empty[s], 1);
@@ -849,6 +846,11 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // everything above overlaps the tail of the preceding kernel; the plan and
+  // the caller's buffers are only touched from here on
+  grid_dependency_wait();
+  grid_launch_dependents();
+  if (misaligned && threadIdx.x == 0) atomicOr(p.err, kErrInternal);
   const uint32_t tmem_base = *tmem_slot;
   const Partition part = load_partition(p);
   if (threadIdx.x == 0) MLA_TRACE_EV(10, 0);
@@ -890,9 +892,8 @@ cudaError_t launch_one(const DecodeParams& p, const CUtensorMap& tkv, int row_ti
     if (e != cudaSuccess) return e;
     __atomic_fetch_or(&configured, bit, __ATOMIC_RELEASE);
   }
-  dim3 grid(p.num_parts, row_tiles);
-  mla_decode_kernel<FP8><<<grid, FP8 ? 320 : 192, smem, stream>>>(p, tkv);
-  return cudaGetLastError();
+  return launch_dependent(mla_decode_kernel<FP8>, dim3(p.num_parts, row_tiles), dim3(FP8 ? 320 : 192), smem, stream,
+                          p, tkv);
 }
 
 }  // namespace

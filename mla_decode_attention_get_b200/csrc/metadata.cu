@@ -14,6 +14,7 @@
 // per boundary, and two scans that turn the distinct interior cut points into
 // split counts and split indices.
 #include "mla_kernels.cuh"
+#include "ptx_sm100.cuh"
 
 namespace mla {
 namespace {
@@ -48,6 +49,8 @@ __global__ void __launch_bounds__(kMdThreads, 1)
                     int* __restrict__ ns) {
   __shared__ int buf[kMdThreads];
   const int tid = threadIdx.x;
+  grid_dependency_wait();        // the previous decode may still read num_splits
+  grid_launch_dependents();
 
   // 1. exclusive prefix of unit costs -> ns[0..U-1] (temporarily), ns[U] = T.
   int carry = 0;
@@ -150,14 +153,149 @@ __global__ void __launch_bounds__(kMdThreads, 1)
   }
 }
 
+// Shared-memory variant for plans whose arrays fit on chip (the common case):
+// the same plan, with the prefix arrays and boundaries kept in shared memory
+// and warp-shuffle scans, so the binary searches never touch global memory.
+constexpr int kMdFastThreads = 1024;
+constexpr int kMdFastMaxInts = 48 * 1024;   // 192 KB of shared memory
+
+// Exclusive block scan of one value per thread (kMdFastThreads threads);
+// returns the exclusive prefix and the block total.
+__device__ __forceinline__ int block_scan_fast(int v, int* warp_sums, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_sums[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += y;
+    }
+    warp_sums[lane] = w;
+  }
+  __syncthreads();
+  const int before = warp > 0 ? warp_sums[warp - 1] : 0;
+  total = warp_sums[31];
+  __syncthreads();
+  return before + x - v;
+}
+
+__global__ void __launch_bounds__(kMdFastThreads, 1)
+    metadata_smem_kernel(const int* __restrict__ seqlens, int s_q, int topk, int U, int P, int* __restrict__ md,
+                         int* __restrict__ ns) {
+  extern __shared__ int sh[];
+  __shared__ int warp_sums[32];
+  int* C = sh;                 // [U + 1] exclusive cost prefix
+  int* NE = C + (U + 1);       // [U + 1] non-empty units before u
+  int* bu = NE + (U + 1);      // [P + 1] boundary unit
+  int* bj = bu + (P + 1);      // [P + 1] boundary page
+  int* F = bj + (P + 1);       // [P + 1] inclusive prefix of cut flags
+  const int tid = threadIdx.x;
+  grid_dependency_wait();        // the previous decode may still read num_splits
+  grid_launch_dependents();
+
+  int carry_c = 0, carry_n = 0;
+  for (int base = 0; base < U; base += kMdFastThreads) {
+    const int u = base + tid;
+    const int n = u < U ? unit_pages(seqlens, u, s_q, topk) : 0;
+    int tc, tn;
+    const int ec = block_scan_fast(n > 0 ? n + kFixedSplitCost : 0, warp_sums, tc);
+    const int en = block_scan_fast(n > 0 ? 1 : 0, warp_sums, tn);
+    if (u < U) { C[u] = carry_c + ec; NE[u] = carry_n + en; }
+    carry_c += tc;
+    carry_n += tn;
+  }
+  if (tid == 0) { C[U] = carry_c; NE[U] = carry_n; }
+  __syncthreads();
+  const long long T = carry_c;
+
+  for (int p = tid; p <= P; p += kMdFastThreads) {
+    const long long x = (static_cast<long long>(p) * T) / P;
+    int b_u = U, b_j = 0;
+    if (x < T) {
+      int lo = 0, hi = U - 1;  // largest u with C[u] <= x
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (static_cast<long long>(C[mid]) <= x) lo = mid; else hi = mid - 1;
+      }
+      b_u = lo;
+      const long long j = x - C[lo] - kFixedSplitCost;
+      b_j = j > 0 ? static_cast<int>(j) : 0;
+    }
+    bu[p] = b_u;
+    bj[p] = b_j;
+  }
+  __syncthreads();
+
+  int carry = 0;
+  for (int base = 0; base < P; base += kMdFastThreads) {
+    const int p = base + tid;
+    int flag = 0;
+    if (p >= 1 && p < P) flag = (bu[p] < U && bj[p] > 0 && (bu[p] != bu[p - 1] || bj[p] != bj[p - 1])) ? 1 : 0;
+    int tf;
+    const int ef = block_scan_fast(flag, warp_sums, tf);
+    if (p < P) F[p] = carry + ef + flag;
+    carry += tf;
+  }
+  __syncthreads();
+
+  // num_splits[u] = NE(u) + (cut flags of units before u)
+  for (int u = tid; u <= U; u += kMdFastThreads) {
+    int lo = 0, hi = P;  // first p in [0, P] with bu[p] >= u
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (bu[mid] >= u) hi = mid; else lo = mid + 1;
+    }
+    ns[u] = NE[u] + (lo > 0 ? F[lo - 1] : 0);
+  }
+  for (int p = tid; p < P; p += kMdFastThreads) {
+    const int u = bu[p];
+    int* row = md + p * kMdWords;
+    row[0] = u;
+    row[1] = bj[p];
+    row[2] = bu[p + 1];
+    row[3] = bj[p + 1];
+    row[4] = u < U ? NE[u] + F[p] : NE[U] + F[P - 1];
+    row[5] = 0;
+    row[6] = 0;
+    row[7] = 0;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_metadata(const int* seqlens, int batch, int s_q, int topk, int num_units, int num_parts,
                             int* tile_md, int* num_splits, int* err, cudaStream_t stream) {
   (void)batch;
   (void)err;
-  metadata_kernel<<<1, kMdThreads, 0, stream>>>(seqlens, s_q, topk, num_units, num_parts, tile_md, num_splits);
-  return cudaGetLastError();
+  const long long ints = 2LL * (num_units + 1) + 3LL * (num_parts + 1);
+  if (ints <= kMdFastMaxInts) {
+    const size_t bytes = static_cast<size_t>(ints) * sizeof(int);
+    if (bytes > 48 * 1024) {
+      static unsigned long long configured = 0;
+      int dev = 0;
+      cudaError_t e = cudaGetDevice(&dev);
+      if (e != cudaSuccess) return e;
+      const unsigned long long bit = 1ull << (dev & 63);
+      if (!(__atomic_load_n(&configured, __ATOMIC_ACQUIRE) & bit)) {
+        e = cudaFuncSetAttribute(metadata_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kMdFastMaxInts * static_cast<int>(sizeof(int)));
+        if (e != cudaSuccess) return e;
+        __atomic_fetch_or(&configured, bit, __ATOMIC_RELEASE);
+      }
+    }
+    return launch_dependent(metadata_smem_kernel, dim3(1), dim3(kMdFastThreads), bytes, stream, seqlens, s_q, topk,
+                            num_units, num_parts, tile_md, num_splits);
+  }
+  return launch_dependent(metadata_kernel, dim3(1), dim3(kMdThreads), 0, stream, seqlens, s_q, topk, num_units,
+                          num_parts, tile_md, num_splits);
 }
 
 }  // namespace mla

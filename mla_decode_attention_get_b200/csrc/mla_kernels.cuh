@@ -5,6 +5,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <utility>
+
 namespace mla {
 
 constexpr int kPage = 64;
@@ -48,6 +50,25 @@ struct DecodeParams {
   float scale_log2;           // softmax_scale * log2(e)
   int causal;
 };
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the preceding kernel of the stream drains; it calls grid_dependency_wait()
+// before touching memory that kernel reads or writes.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Launchers (return cudaSuccess or the launch error).
 cudaError_t launch_metadata(const int* seqlens, int batch, int s_q, int topk, int num_units, int num_parts,

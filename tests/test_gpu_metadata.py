@@ -51,6 +51,16 @@ def test_large_batch_and_single_sequence():
     np.testing.assert_array_equal(ns, np.array(ref_ns))
 
 
+def test_plan_too_large_for_shared_memory():
+    # 2 x 30001 + 3 x 1185 ints exceed the on-chip variant: the global-memory kernel runs
+    rng = np.random.default_rng(7)
+    L = rng.integers(0, 5000, size=30000)
+    md, ns = _gpu_plan(L.tolist(), 1, 16, 0, 1184)
+    ref_md, ref_ns = R.schedule(R.unit_tiles(L), 1184)
+    np.testing.assert_array_equal(ns, np.array(ref_ns))
+    np.testing.assert_array_equal(md, np.array(ref_md))
+
+
 @pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
 def test_config_plans(cfg):
     from mla_decode_attention_get_b200 import inputs as I
