@@ -330,89 +330,127 @@ __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition
 // ---------------------------------------------------------------------------
 // Warps 6-9 (FP8 sparse path): gather the rows the indices name, dequantise
 // NoPE (e4m3 x per-128 scale) and copy RoPE into the bf16 swizzled page tile.
-// Warp dq owns keys [16 dq, 16 dq + 16) of every tile; lane l converts NoPE
-// bytes [16 l, 16 l + 16) of a row and lanes 0-7 copy its 128 RoPE bytes.
+// Warp dq owns keys [16 dq, 16 dq + 16) of every tile; lane l (< 16) resolves
+// key 16 dq + l (index -> block table -> row).  The next tile's indices and
+// table entries are read, and its rows warmed in L2, while the current tile is
+// converted, 8 rows at a time: lane l converts NoPE dims [8 l, 8 l + 8) and
+// [256 + 8 l, 256 + 8 l + 8) and, for l < 16, RoPE dims [512 + 4 l, +4).
 __device__ __forceinline__ void dequant_role(const DecodeParams& p, const Partition& part, uint8_t* smem,
                                              Bars bars, StageInfo* info, volatile int* abort_flag, int dq) {
   const int lane = threadIdx.x & 31;
-  int t = 0;
+  const int kl = lane & 15;
   bool ok = true;
-  for_each_segment(p, part, [&](int u, int jb, int je) -> bool {
-    const UnitInfo ui = unit_info(p, u);
-    const int* idx_row = p.indices + static_cast<int64_t>(u) * p.topk;
-    for (int j = jb; j < je; ++j) {
-      const int s = t % kStages;
-      if (!mbar_wait(&bars.kv_empty[s], ((t / kStages) & 1) ^ 1, abort_flag)) { ok = false; return false; }
-      uint8_t* stage = smem + Smem::kv_off + s * kPageBytes;
-      uint32_t mask = 0;
+
+  // index of this lane's key in the tile a cursor points at (-1 past topk)
+  auto fetch_pos = [&](const Cursor& c) -> int {
+    if (!c.valid) return -1;
+    const int pos_i = kPage * c.j + 16 * dq + kl;
+    return pos_i < p.topk ? p.indices[static_cast<int64_t>(c.u) * p.topk + pos_i] : -1;
+  };
+  // physical row of a key (phys page, slot) and its validity; flags bad entries
+  auto resolve = [&](const Cursor& c, int pos, int& phys) -> bool {
+    if (!c.valid) return false;
+    const UnitInfo ui = unit_info(p, c.u);
+    bool v = pos >= 0 && pos < ui.L;
+    if (!v && pos != -1 && lane < 16) atomicOr(p.err, kErrIndex);
+    phys = -1;
+    if (v) {
+      phys = page_of(p, ui.b, pos >> 6);
+      if (phys < 0 || phys >= p.num_blocks) {
+        if (lane < 16) atomicOr(p.err, kErrBlockTable);
+        v = false;
+      }
+    }
+    return v;
+  };
+  auto row_ptr = [&](int phys, int pos) -> const uint8_t* {
+    return p.kv + static_cast<int64_t>(phys) * p.kv_block_stride + (pos & 63) * kFp8Row;
+  };
+
+  Cursor cur = cursor_begin(p, part);
+  int pos_c = fetch_pos(cur);
+  int phys_c = -1;
+  bool valid_c = resolve(cur, pos_c, phys_c);
+  int t = 0;
+  while (cur.valid) {
+    const int s = t % kStages;
+    if (!mbar_wait(&bars.kv_empty[s], ((t / kStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
+    Cursor nxt = cur;
+    cursor_next(p, part, nxt);
+    const int pos_n = fetch_pos(nxt);   // in flight while batch 0 converts
+    int phys_n = -1;
+    bool valid_n = false;
+    uint8_t* stage = smem + Smem::kv_off + s * kPageBytes;
 #pragma unroll 1
-      for (int kb = 0; kb < 4; ++kb) {
-        const uint8_t* rows[4];
-        bool valid[4];
+    for (int batch = 0; batch < 2; ++batch) {
+      uint2 n0[8], n1[8], rp[8];
+      float s0[8], s1[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int k = 16 * dq + 4 * kb + e;
-          const int pos_i = kPage * j + k;
-          const int pos = pos_i < p.topk ? idx_row[pos_i] : -1;
-          bool v = pos >= 0 && pos < ui.L;
-          if (!v && pos != -1 && lane == 0) atomicOr(p.err, kErrIndex);
-          int phys = -1;
-          if (v) {
-            phys = page_of(p, ui.b, pos >> 6);
-            if (phys < 0 || phys >= p.num_blocks) {
-              if (lane == 0) atomicOr(p.err, kErrBlockTable);
-              v = false;
-            }
-          }
-          valid[e] = v;
-          rows[e] = v ? p.kv + static_cast<int64_t>(phys) * p.kv_block_stride + (pos & 63) * kFp8Row : nullptr;
-        }
-        uint4 nope[4], rope[4];
-        float scale[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          nope[e] = make_uint4(0, 0, 0, 0);
-          rope[e] = make_uint4(0, 0, 0, 0);
-          scale[e] = 0.f;
-          if (valid[e]) {
-            nope[e] = __ldg(reinterpret_cast<const uint4*>(rows[e] + 16 * lane));
-            scale[e] = __ldg(reinterpret_cast<const float*>(rows[e] + 512 + 4 * (lane >> 3)));
-            if (lane < 8) rope[e] = __ldg(reinterpret_cast<const uint4*>(rows[e] + 528 + 16 * lane));
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int k = 16 * dq + 4 * kb + e;   // token row of the tile
-          const int sw = k & 7;
-          uint32_t w[4] = {nope[e].x, nope[e].y, nope[e].z, nope[e].w};
-          uint32_t o[8];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] & 0xFFFFu), __NV_E4M3);
-            const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] >> 16), __NV_E4M3);
-            const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo));
-            const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hi));
-            o[2 * i] = pack_bf16x2(a.x * scale[e], a.y * scale[e]);
-            o[2 * i + 1] = pack_bf16x2(b.x * scale[e], b.y * scale[e]);
-          }
-          const int c = lane >> 2;           // 64-dim block of this lane's 16 NoPE dims
-          const int ch0 = 2 * (lane & 3);    // first 16-B chunk inside the 128-B row
-          const uint32_t rowa = smem_u32(stage + c * kChunkBytes + k * 128);
-          st_shared_v4(rowa + ((ch0 ^ sw) << 4), make_uint4(o[0], o[1], o[2], o[3]));
-          st_shared_v4(rowa + (((ch0 + 1) ^ sw) << 4), make_uint4(o[4], o[5], o[6], o[7]));
-          if (lane < 8) st_shared_v4(smem_u32(stage + 8 * kChunkBytes + k * 128) + ((lane ^ sw) << 4), rope[e]);
-          if (valid[e]) mask |= 1u << (4 * kb + e);
+      for (int e = 0; e < 8; ++e) {
+        const int ki = 8 * batch + e;
+        const int phys = __shfl_sync(0xffffffffu, phys_c, ki);
+        const int pos = __shfl_sync(0xffffffffu, pos_c, ki);
+        const bool v = __shfl_sync(0xffffffffu, valid_c ? 1 : 0, ki) != 0;
+        n0[e] = n1[e] = rp[e] = make_uint2(0, 0);
+        s0[e] = s1[e] = 0.f;
+        if (v) {
+          const uint8_t* row = row_ptr(phys, pos);
+          n0[e] = __ldg(reinterpret_cast<const uint2*>(row + 8 * lane));
+          n1[e] = __ldg(reinterpret_cast<const uint2*>(row + 256 + 8 * lane));
+          s0[e] = __ldg(reinterpret_cast<const float*>(row + 512 + 4 * (lane >> 4)));
+          s1[e] = __ldg(reinterpret_cast<const float*>(row + 520 + 4 * (lane >> 4)));
+          if (lane < 16) rp[e] = __ldg(reinterpret_cast<const uint2*>(row + 528 + 8 * lane));
         }
       }
-      if (lane == 0) info[s].mask[dq] = static_cast<uint16_t>(mask);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.kv_full[s]);
-      ++t;
+      if (batch == 0) {
+        // the next tile's rows: resolve them and warm L2 while batch 1 converts
+        valid_n = resolve(nxt, pos_n, phys_n);
+        if (valid_n && lane < 16) bulk_prefetch_l2(row_ptr(phys_n, pos_n), kFp8Row);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int k = 16 * dq + 8 * batch + e;   // token row of the tile
+        const int sw = k & 7;
+        const uint32_t slot = static_cast<uint32_t>(((lane & 7) ^ sw) << 4);
+        const uint32_t rowa = smem_u32(stage + k * 128);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const uint2 codes = half ? n1[e] : n0[e];
+          const float sc = half ? s1[e] : s0[e];
+          const uint32_t w[2] = {codes.x, codes.y};
+          uint32_t o[4];
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] & 0xFFFFu), __NV_E4M3);
+            const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] >> 16), __NV_E4M3);
+            const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&lo));
+            const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+            o[2 * i] = pack_bf16x2(fa.x * sc, fa.y * sc);
+            o[2 * i + 1] = pack_bf16x2(fb.x * sc, fb.y * sc);
+          }
+          const int chunk = 4 * half + (lane >> 3);
+          st_shared_v4(rowa + chunk * kChunkBytes + slot, make_uint4(o[0], o[1], o[2], o[3]));
+        }
+        if (lane < 16) {
+          const uint32_t unit = static_cast<uint32_t>(((lane >> 1) ^ sw) << 4) + (lane & 1) * 8;
+          asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(rowa + 8 * kChunkBytes + unit), "r"(rp[e].x),
+                       "r"(rp[e].y)
+                       : "memory");
+        }
+      }
     }
-    return true;
-  });
-  if (!ok) raise_abort(abort_flag, p.err);
+    const uint32_t mask = __ballot_sync(0xffffffffu, valid_c) & 0xFFFFu;
+    if (lane == 0) info[s].mask[dq] = static_cast<uint16_t>(mask);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars.kv_full[s]);
+    cur = nxt;
+    pos_c = pos_n;
+    phys_c = phys_n;
+    valid_c = valid_n;
+    ++t;
+  }
+  if (!ok && lane == 0) raise_abort(abort_flag, p.err);
 }
 
 __device__ __forceinline__ int stage_nvalid(const StageInfo& si, bool fp8) {
