@@ -28,7 +28,7 @@
 //    = 9 boxes of 64 tokens x 64 dims) into the ring and warms L2 a few pages
 //    (and the next query tile) ahead; warp 1 issues the MMAs; warps 2-5 write
 //    each segment's query tile into TMEM, run the online softmax and the
-//    epilogue.  On the FP8 sparse path warps 6-9 gather the indexed rows and
+//    epilogue.  On the FP8 sparse path warps 6-13 gather the indexed rows and
 //    dequantise them into the same bf16 page layout.
 //  * The running max only moves when a page's max exceeds it by more than
 //    2^8 (per row); the final division by the row sum uses the same stale
@@ -89,6 +89,9 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemQCol = 128;           // Q tile columns 128..415 in lanes 16-31
 
 constexpr int kWarpLoad = 0, kWarpMma = 1, kWarpSoftmax0 = 2, kWarpDequant0 = 6;
+constexpr int kDequantWarps = 8;              // FP8 path: warp dq converts keys [8 dq, 8 dq + 8)
+constexpr int kThreadsDense = 32 * kWarpDequant0;
+constexpr int kThreadsFp8 = 32 * (kWarpDequant0 + kDequantWarps);
 
 struct Smem {
   static constexpr int kv_off = 0;                               // page ring
@@ -328,66 +331,83 @@ __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition
 }
 
 // ---------------------------------------------------------------------------
-// Warps 6-9 (FP8 sparse path): gather the rows the indices name, dequantise
+// Warps 6-13 (FP8 sparse path): gather the rows the indices name, dequantise
 // NoPE (e4m3 x per-128 scale) and copy RoPE into the bf16 swizzled page tile.
-// Warp dq owns keys [16 dq, 16 dq + 16) of every tile; lane l (< 16) resolves
-// key 16 dq + l (index -> block table -> row).  The next tile's indices and
-// table entries are read, and its rows warmed in L2, while the current tile is
-// converted, 8 rows at a time: lane l converts NoPE dims [8 l, 8 l + 8) and
-// [256 + 8 l, 256 + 8 l + 8) and, for l < 16, RoPE dims [512 + 4 l, +4).
+// Warp dq owns keys [8 dq, 8 dq + 8) of every tile; lane l (< 8) resolves key
+// 8 dq + l (index -> block table -> row).  The next tile's table entries and
+// the index after it are read, and the next rows warmed in L2, while the
+// current tile converts: lane l converts NoPE dims [8 l, 8 l + 8) and
+// [256 + 8 l, 256 + 8 l + 8) and, for l < 16, RoPE dims [512 + 4 l, +4) of
+// each of the warp's 8 rows.
 __device__ __forceinline__ void dequant_role(const DecodeParams& p, const Partition& part, uint8_t* smem,
                                              Bars bars, StageInfo* info, volatile int* abort_flag, int dq) {
   const int lane = threadIdx.x & 31;
-  const int kl = lane & 15;
+  const int kl = lane & 7;
   bool ok = true;
 
   // index of this lane's key in the tile a cursor points at (-1 past topk)
   auto fetch_pos = [&](const Cursor& c) -> int {
     if (!c.valid) return -1;
-    const int pos_i = kPage * c.j + 16 * dq + kl;
+    const int pos_i = kPage * c.j + 8 * dq + kl;
     return pos_i < p.topk ? p.indices[static_cast<int64_t>(c.u) * p.topk + pos_i] : -1;
-  };
-  // physical row of a key (phys page, slot) and its validity; flags bad entries
-  auto resolve = [&](const Cursor& c, int pos, int& phys) -> bool {
-    if (!c.valid) return false;
-    const UnitInfo ui = unit_info(p, c.u);
-    bool v = pos >= 0 && pos < ui.L;
-    if (!v && pos != -1 && lane < 16) atomicOr(p.err, kErrIndex);
-    phys = -1;
-    if (v) {
-      phys = page_of(p, ui.b, pos >> 6);
-      if (phys < 0 || phys >= p.num_blocks) {
-        if (lane < 16) atomicOr(p.err, kErrBlockTable);
-        v = false;
-      }
-    }
-    return v;
   };
   auto row_ptr = [&](int phys, int pos) -> const uint8_t* {
     return p.kv + static_cast<int64_t>(phys) * p.kv_block_stride + (pos & 63) * kFp8Row;
   };
 
+  // Loads behind resolving a tile: the length of its unit and the table entry
+  // of this lane's key, issued together (the entry speculatively).
+  struct Pending {
+    int pos, L, page_entry;
+  };
+  auto start_resolve = [&](const Cursor& c, int pos) -> Pending {
+    Pending r{pos, 0, -1};
+    if (!c.valid) return r;
+    const UnitInfo ui = unit_info(p, c.u);
+    r.L = ui.L;
+    if (pos >= 0) r.page_entry = page_of(p, ui.b, pos >> 6);
+    return r;
+  };
+  auto finish_resolve = [&](const Cursor& c, const Pending& r, int& phys) -> bool {
+    phys = -1;
+    if (!c.valid) return false;
+    bool v = r.pos >= 0 && r.pos < r.L;
+    if (!v && r.pos != -1 && lane < 8) atomicOr(p.err, kErrIndex);
+    if (v) {
+      phys = r.page_entry;
+      if (phys < 0 || phys >= p.num_blocks) {
+        if (lane < 8) atomicOr(p.err, kErrBlockTable);
+        v = false;
+      }
+    }
+    return v;
+  };
+
   Cursor cur = cursor_begin(p, part);
+  Cursor nxt = cur;
+  cursor_next(p, part, nxt);
   int pos_c = fetch_pos(cur);
   int phys_c = -1;
-  bool valid_c = resolve(cur, pos_c, phys_c);
+  bool valid_c = finish_resolve(cur, start_resolve(cur, pos_c), phys_c);
+  int pos_n = fetch_pos(nxt);
   int t = 0;
   while (cur.valid) {
     const int s = t % kStages;
     if (!mbar_wait(&bars.kv_empty[s], ((t / kStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
-    Cursor nxt = cur;
-    cursor_next(p, part, nxt);
-    const int pos_n = fetch_pos(nxt);   // in flight while batch 0 converts
+    if (lane == 0 && dq == 0) MLA_TRACE_EV(0, t);
+    Cursor nxt2 = nxt;
+    cursor_next(p, part, nxt2);
+    const int pos_nn = fetch_pos(nxt2);            // tile t+2: in flight for a whole tile
+    const Pending pend = start_resolve(nxt, pos_n);  // tile t+1: in flight while this tile converts
     int phys_n = -1;
     bool valid_n = false;
     uint8_t* stage = smem + Smem::kv_off + s * kPageBytes;
-#pragma unroll 1
-    for (int batch = 0; batch < 2; ++batch) {
+    {
       uint2 n0[8], n1[8], rp[8];
       float s0[8], s1[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const int ki = 8 * batch + e;
+        const int ki = e;
         const int phys = __shfl_sync(0xffffffffu, phys_c, ki);
         const int pos = __shfl_sync(0xffffffffu, pos_c, ki);
         const bool v = __shfl_sync(0xffffffffu, valid_c ? 1 : 0, ki) != 0;
@@ -402,14 +422,10 @@ __device__ __forceinline__ void dequant_role(const DecodeParams& p, const Partit
           if (lane < 16) rp[e] = __ldg(reinterpret_cast<const uint2*>(row + 528 + 8 * lane));
         }
       }
-      if (batch == 0) {
-        // the next tile's rows: resolve them and warm L2 while batch 1 converts
-        valid_n = resolve(nxt, pos_n, phys_n);
-        if (valid_n && lane < 16) bulk_prefetch_l2(row_ptr(phys_n, pos_n), kFp8Row);
-      }
+      if (lane == 0 && dq == 0) MLA_TRACE_EV(1, t);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const int k = 16 * dq + 8 * batch + e;   // token row of the tile
+        const int k = 8 * dq + e;   // token row of the tile
         const int sw = k & 7;
         const uint32_t slot = static_cast<uint32_t>(((lane & 7) ^ sw) << 4);
         const uint32_t rowa = smem_u32(stage + k * 128);
@@ -439,15 +455,21 @@ __device__ __forceinline__ void dequant_role(const DecodeParams& p, const Partit
         }
       }
     }
-    const uint32_t mask = __ballot_sync(0xffffffffu, valid_c) & 0xFFFFu;
-    if (lane == 0) info[s].mask[dq] = static_cast<uint16_t>(mask);
+    // tile t+1 resolved: warm its rows in L2
+    valid_n = finish_resolve(nxt, pend, phys_n);
+    if (valid_n && lane < 8) bulk_prefetch_l2(row_ptr(phys_n, pos_n), kFp8Row);
+    const uint32_t mask = __ballot_sync(0xffffffffu, valid_c) & 0xFFu;
+    if (lane == 0) reinterpret_cast<uint8_t*>(info[s].mask)[dq] = static_cast<uint8_t>(mask);
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars.kv_full[s]);
+    if (lane == 0 && dq == 0) MLA_TRACE_EV(15, t);
     cur = nxt;
+    nxt = nxt2;
     pos_c = pos_n;
     phys_c = phys_n;
     valid_c = valid_n;
+    pos_n = pos_nn;
     ++t;
   }
   if (!ok && lane == 0) raise_abort(abort_flag, p.err);
@@ -581,44 +603,21 @@ __device__ __forceinline__ void write_q_tile(const DecodeParams& p, const UnitIn
                                              int half) {
   const bool valid = r < tile_valid_rows(p);
   const uint4* src = reinterpret_cast<const uint4*>(p.q + q_tile_offset(p, ui) + static_cast<int64_t>(r) * kDqk);
-  uint4 buf[18];
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    uint4 buf[8];
 #pragma unroll
-  for (int c = 0; c < 2; ++c)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) buf[8 * c + i] = valid ? __ldg(src + 16 * c + 8 * half + i) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-  for (int c = 0; c < 2; ++c) {
+    for (int i = 0; i < 8; ++i) buf[i] = valid ? __ldg(src + 16 * c + 8 * half + i) : make_uint4(0, 0, 0, 0);
     uint32_t v[32];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      v[4 * i] = buf[8 * c + i].x; v[4 * i + 1] = buf[8 * c + i].y;
-      v[4 * i + 2] = buf[8 * c + i].z; v[4 * i + 3] = buf[8 * c + i].w;
-    }
-    tmem_st_16x32bx2_x32u(tq_lane + 64 * c, v);
-  }
-#pragma unroll
-  for (int c = 2; c < 4; ++c)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) buf[8 * (c - 2) + i] = valid ? __ldg(src + 16 * c + 8 * half + i) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-  for (int i = 0; i < 2; ++i) buf[16 + i] = valid ? __ldg(src + 64 + 4 * half + i) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-  for (int c = 2; c < 4; ++c) {
-    uint32_t v[32];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[4 * i] = buf[8 * (c - 2) + i].x; v[4 * i + 1] = buf[8 * (c - 2) + i].y;
-      v[4 * i + 2] = buf[8 * (c - 2) + i].z; v[4 * i + 3] = buf[8 * (c - 2) + i].w;
+      v[4 * i] = buf[i].x; v[4 * i + 1] = buf[i].y; v[4 * i + 2] = buf[i].z; v[4 * i + 3] = buf[i].w;
     }
     tmem_st_16x32bx2_x32u(tq_lane + 64 * c, v);
   }
   uint32_t w[16];
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    w[4 * i] = buf[16 + i].x; w[4 * i + 1] = buf[16 + i].y; w[4 * i + 2] = buf[16 + i].z; w[4 * i + 3] = buf[16 + i].w;
-  }
-#pragma unroll
-  for (int i = 2; i < 4; ++i) {
+  for (int i = 0; i < 4; ++i) {
     const uint4 x = valid ? __ldg(src + 64 + 4 * half + i) : make_uint4(0, 0, 0, 0);
     w[4 * i] = x.x; w[4 * i + 1] = x.y; w[4 * i + 2] = x.z; w[4 * i + 3] = x.w;
   }
@@ -837,7 +836,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
 
 // ---------------------------------------------------------------------------
 template <bool FP8>
-__global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
+__global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreadsDense, 1)
     mla_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_kv) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
@@ -861,7 +860,7 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
   if (threadIdx.x == 0) {
     *abort_flag = misaligned ? 1 : 0;
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars.kv_full[s], FP8 ? 4 : 1);
+      mbar_init(&bars.kv_full[s], FP8 ? kDequantWarps : 1);
       mbar_init(&bars.kv_empty[s], 1);
       info[s].nvalid = 0;
       for (int w = 0; w < 4; ++w) info[s].mask[w] = 0;
@@ -930,7 +929,7 @@ cudaError_t launch_one(const DecodeParams& p, const CUtensorMap& tkv, int row_ti
     if (e != cudaSuccess) return e;
     __atomic_fetch_or(&configured, bit, __ATOMIC_RELEASE);
   }
-  return launch_dependent(mla_decode_kernel<FP8>, dim3(p.num_parts, row_tiles), dim3(FP8 ? 320 : 192), smem, stream,
+  return launch_dependent(mla_decode_kernel<FP8>, dim3(p.num_parts, row_tiles), dim3(FP8 ? kThreadsFp8 : kThreadsDense), smem, stream,
                           p, tkv);
 }
 
