@@ -19,8 +19,9 @@ using mla::kPage;
 struct Plan {
   int units;          // sequences (dense) or (sequence, token) pairs (sparse)
   int rows_per_unit;  // s_q * h_q (dense) or h_q (sparse)
-  int tile_rows;      // query rows per CTA
-  int row_tiles;      // CTAs per partition
+  int tile_rows;      // query rows per CTA (per CTA pair on the two-CTA kernel)
+  int row_tiles;      // row tiles per partition
+  bool pair;          // two-CTA kernel
 };
 
 int make_plan(int batch, int s_q, int h_q, int h_kv, int topk, Plan* pl) {
@@ -31,7 +32,8 @@ int make_plan(int batch, int s_q, int h_q, int h_kv, int topk, Plan* pl) {
   if (rows > (1 << 20) || units > (1 << 24)) return MLA_ERR_INVALID_ARG;
   pl->units = static_cast<int>(units);
   pl->rows_per_unit = topk > 0 ? h_q : static_cast<int>(rows);
-  pl->tile_rows = mla::tile_rows_for(pl->rows_per_unit);
+  pl->pair = mla::use_pair_kernel(pl->rows_per_unit, topk > 0);
+  pl->tile_rows = mla::tile_rows_for(pl->rows_per_unit, topk > 0);
   pl->row_tiles = (pl->rows_per_unit + pl->tile_rows - 1) / pl->tile_rows;
   return MLA_OK;
 }
@@ -51,11 +53,17 @@ int device_sm_count(int* out) {
   return MLA_OK;
 }
 
+size_t lse_region_bytes(const Plan& pl, int num_parts) {
+  const size_t splits = static_cast<size_t>(pl.units) + static_cast<size_t>(num_parts);
+  return (splits * pl.rows_per_unit * sizeof(float) + 255) & ~size_t(255);
+}
+
 size_t workspace_need(const Plan& pl, int num_parts) {
   const size_t splits = static_cast<size_t>(pl.units) + static_cast<size_t>(num_parts);
   const size_t o_bytes = splits * pl.rows_per_unit * kDv * sizeof(float);
-  const size_t l_bytes = splits * pl.rows_per_unit * sizeof(float);
-  return o_bytes + ((l_bytes + 255) & ~size_t(255));
+  const size_t ring = pl.pair ? static_cast<size_t>(num_parts) * pl.row_tiles * mla::kPairSlots * mla::kPairSlotBytes
+                              : 0;
+  return o_bytes + lse_region_bytes(pl, num_parts) + ring;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -134,6 +142,7 @@ int prepare(const mla_decode_args* a, Plan* pl, mla::DecodeParams* kp) {
   const size_t splits = static_cast<size_t>(pl->units) + static_cast<size_t>(a->num_parts);
   kp->ws_o = static_cast<float*>(a->workspace);
   kp->ws_lse = kp->ws_o + splits * pl->rows_per_unit * kDv;
+  kp->ws_pring = pl->pair ? reinterpret_cast<uint8_t*>(kp->ws_lse) + lse_region_bytes(*pl, a->num_parts) : nullptr;
   kp->err = a->err_word;
   kp->batch = a->batch;
   kp->s_q = a->s_q;
@@ -159,7 +168,10 @@ int mla_metadata_shape(int batch, int s_q, int h_q, int h_kv, int topk, int num_
     int sms = 0;
     st = device_sm_count(&sms);
     if (st != MLA_OK) return st;
-    parts = sms / pl.row_tiles;
+    // one partition per SM (per row tile), or per co-resident CTA pair
+    const int slots = pl.pair ? mla::pair_cluster_capacity() : sms;
+    if (slots < 1) return MLA_ERR_CUDA;
+    parts = slots / pl.row_tiles;
     if (parts < 1) parts = 1;
   }
   if (parts > (1 << 16)) return MLA_ERR_INVALID_ARG;
@@ -199,7 +211,8 @@ int mla_decode_attention(const mla_decode_args* a, void* stream) {
                                      uint64_t(kDqk) * 2, uint64_t(a->k_block_stride), kPage))
     return MLA_ERR_CUDA;
   const cudaError_t e =
-      mla::launch_decode(kp, tkv, pl.tile_rows, a->is_fp8 != 0, pl.row_tiles, static_cast<cudaStream_t>(stream));
+      pl.pair ? mla::launch_decode_pair(kp, tkv, pl.row_tiles, static_cast<cudaStream_t>(stream))
+              : mla::launch_decode(kp, tkv, pl.tile_rows, a->is_fp8 != 0, pl.row_tiles, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

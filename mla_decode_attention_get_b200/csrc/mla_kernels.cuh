@@ -17,12 +17,22 @@ constexpr int kFp8Row = 656;
 constexpr int kMdWords = 8;
 constexpr int kFixedSplitCost = 5;
 
-// Row tile of the decode kernel: the number of (token, head) query rows a CTA
-// handles (the M of every tensor-core MMA); units with fewer rows leave the
-// rest of the tile as zero padding.
-__host__ __device__ constexpr int tile_rows_for(int rows_per_unit) {
-  return (void)rows_per_unit, 64;
+// Row tile of the decode: the number of (token, head) query rows one CTA (or
+// one CTA pair) handles, the M of every tensor-core MMA; units with fewer
+// rows leave the rest of the tile as zero padding.  Dense units of more than
+// 64 rows run on the two-CTA kernel with 128-row tiles.
+__host__ __device__ constexpr bool use_pair_kernel(int rows_per_unit, bool sparse) {
+  return !sparse && rows_per_unit > 64;
 }
+__host__ __device__ constexpr int tile_rows_for(int rows_per_unit, bool sparse) {
+  return use_pair_kernel(rows_per_unit, sparse) ? 128 : 64;
+}
+
+// Two-CTA kernel: per cluster, a ring of kPairSlots entries in global memory
+// carries P [128 x 64] bf16, alpha[128] and 1/l[128] from the score CTA to
+// the value CTA.
+constexpr int kPairSlots = 4;
+constexpr int kPairSlotBytes = 128 * 128 + 2 * 128 * 4;   // 17408
 
 struct DecodeParams {
   const uint16_t* q;          // bf16 bits [batch, s_q, h_q, 576]
@@ -44,6 +54,7 @@ struct DecodeParams {
   float* lse;
   float* ws_o;                // [splits, rows_per_unit, 512]
   float* ws_lse;              // [splits, rows_per_unit]
+  uint8_t* ws_pring;          // two-CTA kernel: [clusters, kPairSlots, kPairSlotBytes]
   int* err;
   int batch, s_q, h_q;
   int rows_per_unit;
@@ -76,6 +87,11 @@ cudaError_t launch_metadata(const int* seqlens, int batch, int s_q, int topk, in
 
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, int tile_rows, bool fp8, int row_tiles,
                           cudaStream_t stream);
+
+cudaError_t launch_decode_pair(const DecodeParams& p, const CUtensorMap& tmap_kv, int row_tiles, cudaStream_t stream);
+
+// Clusters of the two-CTA kernel that fit on the current device at once.
+int pair_cluster_capacity();
 
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream);
 

@@ -67,6 +67,12 @@ def test_workspace_bytes(lib):
     n = _abi.workspace_bytes(64, 1, 128, 2048, 74)
     splits = 64 + 74
     assert n == splits * 128 * 512 * 4 + ((splits * 128 * 4 + 255) // 256) * 256
+    # dense units of more than 64 rows (two-CTA kernel) add, per partition and
+    # 128-row tile, a ring of 4 entries of P [128 x 64] bf16 + 2 x 128 floats
+    n = _abi.workspace_bytes(132, 2, 128, 0, 37)
+    splits = 132 + 37
+    ring = 37 * 2 * 4 * (128 * 128 + 2 * 128 * 4)
+    assert n == splits * 256 * 512 * 4 + ((splits * 256 * 4 + 255) // 256) * 256 + ring
 
 
 def test_decode_rejects_bad_arguments_before_launch(lib):
