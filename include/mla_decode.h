@@ -131,7 +131,7 @@ typedef struct mla_decode_args {
   size_t workspace_bytes;       /* >= mla_workspace_bytes() */
   int32_t* err_word;            /* int32, caller-zeroed; MLA_DEVERR_* bits (output) */
   int32_t batch, s_q, h_q, h_kv, d_v;
-  float softmax_scale;          /* logits = softmax_scale * q.k */
+  float softmax_scale;          /* logits = softmax_scale * q.k; finite and > 0 */
   int32_t causal;               /* dense s_q > 1: token i sees keys t <= L - s_q + i */
   int32_t is_fp8;               /* k_cache holds FP8 rows (requires indices) */
 } mla_decode_args;

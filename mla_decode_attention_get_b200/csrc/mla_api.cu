@@ -5,6 +5,7 @@
 
 #include <atomic>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 
 #include "mla_decode.h"
@@ -24,6 +25,14 @@ struct Plan {
   bool pair;          // two-CTA kernel
 };
 
+// MLA_TWO_CTA_DECODE=1 in the environment selects the two-CTA kernel for
+// dense units of more than 64 rows (read on every call; the metadata,
+// workspace and decode calls of one step must see the same value).
+bool two_cta_opt_in() {
+  const char* v = std::getenv("MLA_TWO_CTA_DECODE");
+  return v != nullptr && v[0] == '1' && v[1] == '\0';
+}
+
 int make_plan(int batch, int s_q, int h_q, int h_kv, int topk, Plan* pl) {
   if (batch < 1 || s_q < 1 || h_q < 1 || topk < 0) return MLA_ERR_INVALID_ARG;
   if (h_kv != 1) return MLA_ERR_UNSUPPORTED;
@@ -32,8 +41,9 @@ int make_plan(int batch, int s_q, int h_q, int h_kv, int topk, Plan* pl) {
   if (rows > (1 << 20) || units > (1 << 24)) return MLA_ERR_INVALID_ARG;
   pl->units = static_cast<int>(units);
   pl->rows_per_unit = topk > 0 ? h_q : static_cast<int>(rows);
-  pl->pair = mla::use_pair_kernel(pl->rows_per_unit, topk > 0);
-  pl->tile_rows = mla::tile_rows_for(pl->rows_per_unit, topk > 0);
+  const bool opt_in = two_cta_opt_in();
+  pl->pair = mla::use_pair_kernel(pl->rows_per_unit, topk > 0, opt_in);
+  pl->tile_rows = mla::tile_rows_for(pl->rows_per_unit, topk > 0, opt_in);
   pl->row_tiles = (pl->rows_per_unit + pl->tile_rows - 1) / pl->tile_rows;
   return MLA_OK;
 }
@@ -118,7 +128,7 @@ int prepare(const mla_decode_args* a, Plan* pl, mla::DecodeParams* kp) {
   if (a->k_block_stride < page_bytes || a->k_block_stride % 16 != 0) return MLA_ERR_INVALID_ARG;
   const int64_t rows = int64_t(a->s_q) * a->h_q;
   if (a->q_batch_stride < rows * kDqk || a->q_batch_stride % 8 != 0) return MLA_ERR_INVALID_ARG;
-  if (!std::isfinite(a->softmax_scale)) return MLA_ERR_INVALID_ARG;
+  if (!std::isfinite(a->softmax_scale) || !(a->softmax_scale > 0.f)) return MLA_ERR_INVALID_ARG;
   if (a->workspace_bytes < workspace_need(*pl, a->num_parts)) return MLA_ERR_WORKSPACE;
 
   std::memset(kp, 0, sizeof(*kp));

@@ -19,19 +19,22 @@ constexpr int kFixedSplitCost = 5;
 
 // Row tile of the decode: the number of (token, head) query rows one CTA (or
 // one CTA pair) handles, the M of every tensor-core MMA; units with fewer
-// rows leave the rest of the tile as zero padding.  Dense units of more than
-// 64 rows run on the two-CTA kernel with 128-row tiles.
-__host__ __device__ constexpr bool use_pair_kernel(int rows_per_unit, bool sparse) {
-  return !sparse && rows_per_unit > 64;
+// rows leave the rest of the tile as zero padding.  The default is the
+// single-CTA kernel with 64-row tiles.  The two-CTA kernel (128-row tiles)
+// serves dense units of more than 64 rows when the caller opts in (it is
+// slower on this hardware today).
+__host__ __device__ constexpr bool use_pair_kernel(int rows_per_unit, bool sparse, bool two_cta_opt_in) {
+  return two_cta_opt_in && !sparse && rows_per_unit > 64;
 }
-__host__ __device__ constexpr int tile_rows_for(int rows_per_unit, bool sparse) {
-  return use_pair_kernel(rows_per_unit, sparse) ? 128 : 64;
+__host__ __device__ constexpr int tile_rows_for(int rows_per_unit, bool sparse, bool two_cta_opt_in) {
+  return use_pair_kernel(rows_per_unit, sparse, two_cta_opt_in) ? 128 : 64;
 }
 
 // Two-CTA kernel: per cluster, a ring of kPairSlots entries in global memory
 // carries P [128 x 64] bf16, alpha[128] and 1/l[128] from the score CTA to
-// the value CTA.
-constexpr int kPairSlots = 4;
+// the value CTA, released and handed back in groups of kPairGroup pages.
+constexpr int kPairGroup = 8;
+constexpr int kPairSlots = 2 * kPairGroup;
 constexpr int kPairSlotBytes = 128 * 128 + 2 * 128 * 4;   // 17408
 
 struct DecodeParams {

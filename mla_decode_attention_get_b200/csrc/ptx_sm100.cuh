@@ -90,6 +90,11 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthread
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Arrive on named barrier `id` without waiting (whole warps).
+__device__ __forceinline__ void named_barrier_arrive(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // ------------------------------------------------------------------ dependent launch
 
 // Wait until the preceding kernel in the stream has completed and its memory
@@ -478,6 +483,22 @@ __device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uin
 // (bulk copy / TMA) reads of them.
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Loads cached in L2 only (data another SM rewrites between reads).
+__device__ __forceinline__ uint4 ld_global_cg_v4(const void* ptr) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(reinterpret_cast<uint64_t>(ptr))
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ float ld_global_cg_f32(const void* ptr) {
+  float v;
+  asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(reinterpret_cast<uint64_t>(ptr)) : "memory");
+  return v;
 }
 
 // Bulk copy of `bytes` (multiple of 16, both addresses 16-B aligned) from

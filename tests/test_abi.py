@@ -67,12 +67,22 @@ def test_workspace_bytes(lib):
     n = _abi.workspace_bytes(64, 1, 128, 2048, 74)
     splits = 64 + 74
     assert n == splits * 128 * 512 * 4 + ((splits * 128 * 4 + 255) // 256) * 256
-    # dense units of more than 64 rows (two-CTA kernel) add, per partition and
-    # 128-row tile, a ring of 4 entries of P [128 x 64] bf16 + 2 x 128 floats
+    base = (132 + 37) * 256 * 512 * 4 + (((132 + 37) * 256 * 4 + 255) // 256) * 256
+    assert _abi.workspace_bytes(132, 2, 128, 0, 37) == base
+
+
+def test_workspace_bytes_two_cta(lib, monkeypatch):
+    # opting in to the two-CTA kernel adds, per partition and 128-row tile of
+    # a dense unit of more than 64 rows, a ring of 16 entries of
+    # P [128 x 64] bf16 + 2 x 128 floats
+    monkeypatch.setenv("MLA_TWO_CTA_DECODE", "1")
     n = _abi.workspace_bytes(132, 2, 128, 0, 37)
     splits = 132 + 37
-    ring = 37 * 2 * 4 * (128 * 128 + 2 * 128 * 4)
+    ring = 37 * 2 * 16 * (128 * 128 + 2 * 128 * 4)
     assert n == splits * 256 * 512 * 4 + ((splits * 256 * 4 + 255) // 256) * 256 + ring
+    # sparse units and units of at most 64 rows keep the single-CTA kernel
+    assert _abi.workspace_bytes(64, 1, 128, 2048, 74) == (64 + 74) * 128 * 2048 + ((138 * 128 * 4 + 255) // 256) * 256
+    assert _abi.workspace_bytes(128, 1, 64, 0, 148) == (128 + 148) * 64 * 2048 + ((276 * 64 * 4 + 255) // 256) * 256
 
 
 def test_decode_rejects_bad_arguments_before_launch(lib):
@@ -113,6 +123,11 @@ def test_decode_checks_alignment_and_workspace(lib):
     a.q = fake
     a.k_block_stride = 64 * 576 * 2 - 16                                    # page overlaps the next
     assert L.mla_decode(ctypes.byref(a), None) == _abi.MLA_ERR_INVALID_ARG
+    a.k_block_stride = 64 * 576 * 2
+    for bad in (0.0, -0.04, float("nan"), float("inf")):                    # softmax_scale finite, > 0
+        a.softmax_scale = bad
+        assert L.mla_decode(ctypes.byref(a), None) == _abi.MLA_ERR_INVALID_ARG
+    a.softmax_scale = 576 ** -0.5
     a.k_block_stride = 64 * 576 * 2
     a.q_batch_stride = 16 * 576 - 8
     assert L.mla_decode(ctypes.byref(a), None) == _abi.MLA_ERR_INVALID_ARG

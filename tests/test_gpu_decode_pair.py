@@ -1,5 +1,6 @@
 """Parity of the two-CTA decode kernel (dense units of more than 64 query
-rows, 128-row tiles) against the fp64 oracle, through the C ABI.
+rows, 128-row tiles; selected by MLA_TWO_CTA_DECODE=1) against the fp64
+oracle, through the C ABI.
 
 The cases aim at what is particular to that kernel: row counts that leave
 part of a 128-row tile empty or need a second tile, causal tiles holding two
@@ -17,11 +18,18 @@ from gpu_util import assert_close, oracle, run
 pytestmark = pytest.mark.gpu
 
 
-def test_pair_kernel_is_selected():
+@pytest.fixture(autouse=True)
+def two_cta(monkeypatch):
+    monkeypatch.setenv("MLA_TWO_CTA_DECODE", "1")
+
+
+def test_pair_kernel_is_selected(monkeypatch):
     # >64 dense rows per unit: partitions are counted in CTA pairs
     parts_pair, _ = M.mla_metadata_shape(4, 1, 128, 1, 0)
     parts_single, _ = M.mla_metadata_shape(4, 1, 64, 1, 0)
     assert parts_pair <= parts_single // 2
+    monkeypatch.delenv("MLA_TWO_CTA_DECODE")
+    assert M.mla_metadata_shape(4, 1, 128, 1, 0)[0] == parts_single // 2   # default: 64-row tiles
 
 
 @pytest.mark.parametrize("h_q,s_q", [(72, 1), (96, 1), (128, 1), (64, 2), (80, 2), (128, 2), (128, 3), (256, 1)])
