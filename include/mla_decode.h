@@ -133,7 +133,11 @@ typedef struct mla_decode_args {
   int32_t batch, s_q, h_q, h_kv, d_v;
   float softmax_scale;          /* logits = softmax_scale * q.k; finite and > 0 */
   int32_t causal;               /* dense s_q > 1: token i sees keys t <= L - s_q + i */
-  int32_t is_fp8;               /* k_cache holds FP8 rows (requires indices) */
+  int32_t is_fp8;               /* k_cache holds FP8 rows (requires indices).  The
+                                   FP8 path dequantises into f16 and runs its
+                                   products on f16 operands (fp32 accumulation):
+                                   dequantised cache values and q must lie
+                                   within +-65504, the f16 range. */
 } mla_decode_args;
 
 /*

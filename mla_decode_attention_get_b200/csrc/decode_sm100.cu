@@ -220,7 +220,9 @@ __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition
 
 // ---------------------------------------------------------------------------
 // Warps 6-13 (FP8 sparse path): gather the rows the indices name, dequantise
-// NoPE (e4m3 x per-128 scale) and copy RoPE into the bf16 swizzled page tile.
+// NoPE (e4m3 x per-128 scale) and convert RoPE into the f16 swizzled page
+// tile (the FP8 path runs its MMAs on f16 operands: the e4m3 codes convert
+// to f16 exactly and one packed multiply applies the scale).
 // Warp dq owns keys [8 dq, 8 dq + 8) of every tile; lane l (< 8) resolves key
 // 8 dq + l (index -> block table -> row).  The next tile's table entries and
 // the index after it are read, and the next rows warmed in L2, while the
@@ -319,26 +321,28 @@ __device__ __forceinline__ void dequant_role(const DecodeParams& p, const Partit
         const uint32_t rowa = smem_u32(stage + k * 128);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
+          // e4m3 pairs convert exactly to f16 pairs; one packed f16 multiply
+          // applies the block scale (rounded once, to 11 significant bits)
           const uint2 codes = half ? n1[e] : n0[e];
           const float sc = half ? s1[e] : s0[e];
+          const uint32_t sc2 = pack_f16x2(sc, sc);
           const uint32_t w[2] = {codes.x, codes.y};
           uint32_t o[4];
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] & 0xFFFFu), __NV_E4M3);
             const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] >> 16), __NV_E4M3);
-            const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&lo));
-            const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&hi));
-            o[2 * i] = pack_bf16x2(fa.x * sc, fa.y * sc);
-            o[2 * i + 1] = pack_bf16x2(fb.x * sc, fb.y * sc);
+            o[2 * i] = hmul2_f16(*reinterpret_cast<const uint32_t*>(&lo), sc2);
+            o[2 * i + 1] = hmul2_f16(*reinterpret_cast<const uint32_t*>(&hi), sc2);
           }
           const int chunk = 4 * half + (lane >> 3);
           st_shared_v4(rowa + chunk * kChunkBytes + slot, make_uint4(o[0], o[1], o[2], o[3]));
         }
         if (lane < 16) {
+          // RoPE dims arrive as bf16: to f16 like the rest of the tile
           const uint32_t unit = static_cast<uint32_t>(((lane >> 1) ^ sw) << 4) + (lane & 1) * 8;
-          asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(rowa + 8 * kChunkBytes + unit), "r"(rp[e].x),
-                       "r"(rp[e].y)
+          asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(rowa + 8 * kChunkBytes + unit),
+                       "r"(bf16x2_to_f16x2(rp[e].x)), "r"(bf16x2_to_f16x2(rp[e].y))
                        : "memory");
         }
       }
@@ -379,8 +383,9 @@ __device__ __forceinline__ int stage_nvalid(const StageInfo& si, bool fp8) {
 template <bool FP8>
 __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition& part, uint8_t* smem, Bars bars,
                                          const StageInfo* info, uint32_t tmem_base, volatile int* abort_flag) {
-  constexpr uint32_t idesc_qk = idesc_bf16_f32(kRows, kPage, false, false);   // S = Q K^T
-  constexpr uint32_t idesc_pv = idesc_bf16_f32(kRows, 256, false, true);      // O += P V (V MN-major)
+  // S = Q K^T and O += P V (V MN-major); the FP8 path runs on f16 operands
+  constexpr uint32_t idesc_qk = FP8 ? idesc_f16_f32(kRows, kPage, false, false) : idesc_bf16_f32(kRows, kPage, false, false);
+  constexpr uint32_t idesc_pv = FP8 ? idesc_f16_f32(kRows, 256, false, true) : idesc_bf16_f32(kRows, 256, false, true);
   const uint32_t tmem_q = tmem_base + (16u << 16) + kTmemQCol;   // A operand of QK (lanes 16-31)
   const uint64_t p_desc = sdesc_sw128(smem_u32(smem + Smem::p_off), 16, 1024);
   uint64_t k_desc[kStages], v_desc[kStages];
@@ -485,8 +490,10 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
 
 // ---------------------------------------------------------------------------
 // Warps 2-5 (whole warps): the query tile of a unit into TMEM lanes 16-31 as
-// packed bf16 pairs.  Thread (r, half) writes row r's dims
-// [128 c + 64 half, +64) for c = 0..3 and RoPE dims [512 + 32 half, +32).
+// packed bf16 pairs (f16 pairs on the FP8 path).  Thread (r, half) writes
+// row r's dims [128 c + 64 half, +64) for c = 0..3 and RoPE dims
+// [512 + 32 half, +32).
+template <bool F16>
 __device__ __forceinline__ void write_q_tile(const DecodeParams& p, const UnitInfo& ui, uint32_t tq_lane, int r,
                                              int half) {
   const bool valid = r < tile_valid_rows(p);
@@ -501,6 +508,10 @@ __device__ __forceinline__ void write_q_tile(const DecodeParams& p, const UnitIn
     for (int i = 0; i < 8; ++i) {
       v[4 * i] = buf[i].x; v[4 * i + 1] = buf[i].y; v[4 * i + 2] = buf[i].z; v[4 * i + 3] = buf[i].w;
     }
+    if (F16) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = bf16x2_to_f16x2(v[i]);
+    }
     tmem_st_16x32bx2_x32u(tq_lane + 64 * c, v);
   }
   uint32_t w[16];
@@ -508,6 +519,10 @@ __device__ __forceinline__ void write_q_tile(const DecodeParams& p, const UnitIn
   for (int i = 0; i < 4; ++i) {
     const uint4 x = valid ? __ldg(src + 64 + 4 * half + i) : make_uint4(0, 0, 0, 0);
     w[4 * i] = x.x; w[4 * i + 1] = x.y; w[4 * i + 2] = x.z; w[4 * i + 3] = x.w;
+  }
+  if (F16) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) w[i] = bf16x2_to_f16x2(w[i]);
   }
   tmem_st_16x32bx2_x16(tq_lane + 256, w);
 }
@@ -541,7 +556,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
     for (int u = u_from; u <= part.u1 && u < p.num_units; ++u) {
       int jb, je;
       if (segment_bounds(p, part, u, jb, je)) {
-        write_q_tile(p, unit_info(p, u), tq_lane, r, half);
+        write_q_tile<FP8>(p, unit_info(p, u), tq_lane, r, half);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bars.q_full);
@@ -630,7 +645,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
           const float a = fast_exp2(x[2 * i] - m_safe);
           const float b = fast_exp2(x[2 * i + 1] - m_safe);
           lsum += a + b;
-          pk[i] = pack_bf16x2(a, b);
+          pk[i] = FP8 ? pack_f16x2(a, b) : pack_bf16x2(a, b);
         }
         l_run += lsum;
       } else {
