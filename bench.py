@@ -120,6 +120,22 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+def max_over_ranks(ms: float, device) -> float:
+    """The slowest rank's time (every rank passes its own; the process group
+    is initialised).  Timing only: the decode itself exchanges nothing."""
+    import torch
+    import torch.distributed as dist
+    x = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(x, op=dist.ReduceOp.MAX)
+    return float(x.item())
+
+
+def whole_job_rates(kv_bytes: int, flops: int, world: int, ms_step: float):
+    """(GB/s, TFLOP/s) of all ranks together: every rank decodes its own
+    batch of the workload in ms_step (the slowest rank's step time)."""
+    return kv_bytes * world / (ms_step * 1e-3) / 1e9, flops * world / (ms_step * 1e-3) / 1e12
+
+
 def _blas_threads() -> int:
     try:
         import threadpoolctl
@@ -292,13 +308,9 @@ def main():
     torch.cuda.synchronize()
     attn_ms = sum(a.elapsed_time(b) for a, b in attn_ev) / args.steps
     if world > 1:
-        import torch.distributed as dist
-        x = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(x, op=dist.ReduceOp.MAX)
-        ms_total = float(x.item())
+        ms_total = max_over_ranks(ms_total, dev)
     ms_step = ms_total / args.steps
-    value = kv_bytes * world / (ms_step * 1e-3) / 1e9
-    tflops = flops * world / (ms_step * 1e-3) / 1e12
+    value, tflops = whole_job_rates(kv_bytes, flops, world, ms_step)
 
     # ---- end to end through the public API, host buffers, copies in the region
     q_host = t["q"].cpu().pin_memory()
