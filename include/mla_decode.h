@@ -59,7 +59,7 @@ extern "C" {
 enum {
   MLA_OK = 0,
   MLA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, bad dim */
-  MLA_ERR_UNSUPPORTED = 2,   /* h_kv != 1, d_v != 512, fp8 without indices ... */
+  MLA_ERR_UNSUPPORTED = 2,   /* h_kv != 1, d_v != 512, indices with a bf16 cache ... */
   MLA_ERR_WORKSPACE = 3,     /* workspace smaller than mla_workspace_bytes() */
   MLA_ERR_CUDA = 4           /* a CUDA runtime call or launch failed */
 };
@@ -133,8 +133,11 @@ typedef struct mla_decode_args {
   int32_t batch, s_q, h_q, h_kv, d_v;
   float softmax_scale;          /* logits = softmax_scale * q.k; finite and > 0 */
   int32_t causal;               /* dense s_q > 1: token i sees keys t <= L - s_q + i */
-  int32_t is_fp8;               /* k_cache holds FP8 rows (requires indices).  The
-                                   FP8 path dequantises into f16 and runs its
+  int32_t is_fp8;               /* k_cache holds FP8 rows: read through indices
+                                   (sparse) or, with indices == NULL, walked page
+                                   by page like the bf16 cache (dense; causal
+                                   applies).  The FP8 path dequantises into f16
+                                   and runs its
                                    products on f16 operands (fp32 accumulation):
                                    dequantised cache values and q must lie
                                    within +-65504, the f16 range. */

@@ -175,7 +175,6 @@ def prepare_decode(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.Te
         if k_cache.dtype != torch.uint8:
             k_cache = k_cache.view(torch.uint8)
         _require(k_cache.shape[-1] == FP8_ROW_BYTES, "fp8 cache rows must be 656 bytes")
-        _require(indices is not None, "the fp8 cache is read through sparse indices")
     else:
         _require(k_cache.dtype == torch.bfloat16 and k_cache.shape[-1] == D_QK, "bf16 cache rows must be 576 wide")
     _require(k_cache[0].is_contiguous(), "each cache page must be contiguous")
@@ -184,6 +183,7 @@ def prepare_decode(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.Te
     _require(cache_seqlens.dtype == torch.int32 and cache_seqlens.is_contiguous(), "cache_seqlens must be int32")
     b, s_q, h_q, _ = q.shape
     if indices is not None:
+        _require(is_fp8_kvcache, "sparse indices are read with the fp8 cache only")
         _require(indices.dtype == torch.int32 and indices.dim() == 3 and indices.shape[:2] == (b, s_q)
                  and indices.is_contiguous(), "indices must be contiguous int32 [batch, s_q, topk]")
     topk = indices.shape[-1] if indices is not None else 0

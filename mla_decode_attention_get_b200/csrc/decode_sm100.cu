@@ -235,10 +235,14 @@ __device__ __forceinline__ void dequant_role(const DecodeParams& p, const Partit
   const int kl = lane & 7;
   bool ok = true;
 
-  // index of this lane's key in the tile a cursor points at (-1 past topk)
+  // Position of this lane's key in the tile a cursor points at: the index
+  // the indices tensor names (-1 past topk), or, with no indices (the dense
+  // FP8 path), the tile's own cache position (positions >= L are padding).
+  const bool sparse = p.indices != nullptr;
   auto fetch_pos = [&](const Cursor& c) -> int {
     if (!c.valid) return -1;
     const int pos_i = kPage * c.j + 8 * dq + kl;
+    if (!sparse) return pos_i;
     return pos_i < p.topk ? p.indices[static_cast<int64_t>(c.u) * p.topk + pos_i] : -1;
   };
   auto row_ptr = [&](int phys, int pos) -> const uint8_t* {
@@ -262,7 +266,7 @@ __device__ __forceinline__ void dequant_role(const DecodeParams& p, const Partit
     phys = -1;
     if (!c.valid) return false;
     bool v = r.pos >= 0 && r.pos < r.L;
-    if (!v && r.pos != -1 && lane < 8) atomicOr(p.err, kErrIndex);
+    if (!v && r.pos != -1 && sparse && lane < 8) atomicOr(p.err, kErrIndex);
     if (v) {
       phys = r.page_entry;
       if (phys < 0 || phys >= p.num_blocks) {
@@ -543,7 +547,8 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
   const float scale_log2 = p.scale_log2;
   const int h_q = p.h_q, s_q = p.s_q;
   const int tok_dense = grow / h_q;                  // dense path: the row's query token
-  const bool causal = !FP8 && p.causal != 0;
+  const bool sparse = p.indices != nullptr;        // (the sparse path is always FP8)
+  const bool causal = !sparse && p.causal != 0;
   const uint32_t s_taddr = tmem_base + (static_cast<uint32_t>(32 * q4 + 16) << 16);
   const uint32_t o_taddr = tmem_base + (static_cast<uint32_t>(32 * q4) << 16);
   const uint32_t p_row = smem_u32(smem + Smem::p_off) + r * 128;
@@ -571,7 +576,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
 
   for_each_segment(p, part, [&](int u, int jb, int je) -> bool {
     const UnitInfo ui = unit_info(p, u);
-    if (!FP8 && lane == 0 && q4 == 0 && p.seqlens[ui.b] < 0) atomicOr(p.err, kErrSeqlen);
+    if (!sparse && lane == 0 && q4 == 0 && p.seqlens[ui.b] < 0) atomicOr(p.err, kErrSeqlen);
     float m_run = -INFINITY, l_run = 0.f;
     bool any_pv = false;
     const int lim = ui.L - s_q + tok_dense + 1;      // causal: keys t < lim are visible
@@ -598,10 +603,10 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
         } else {
           const int nk = min(max(nv - key0, 0), 32);
           vmask = nk >= 32 ? 0xFFFFFFFFu : ((1u << nk) - 1u);
-          if (causal && kPage * j + key0 + 31 >= lim) {
-            const int nc = min(max(lim - kPage * j - key0, 0), 32);
-            vmask &= nc >= 32 ? 0xFFFFFFFFu : ((1u << nc) - 1u);
-          }
+        }
+        if (causal && kPage * j + key0 + 31 >= lim) {
+          const int nc = min(max(lim - kPage * j - key0, 0), 32);
+          vmask &= nc >= 32 ? 0xFFFFFFFFu : ((1u << nc) - 1u);
         }
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -722,7 +727,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
             p.ws_lse[static_cast<int64_t>(split_idx) * R + grow] = lse;
           } else {
             int b, tok, h;
-            if (FP8) { b = ui.b; tok = ui.token; h = grow; }
+            if (sparse) { b = ui.b; tok = ui.token; h = grow; }
             else { b = ui.b; tok = tok_dense; h = grow % h_q; }
             p.lse[(static_cast<int64_t>(b) * h_q + h) * s_q + tok] = lse;
           }

@@ -113,7 +113,7 @@ int prepare(const mla_decode_args* a, Plan* pl, mla::DecodeParams* kp) {
   int st = make_plan(a->batch, a->s_q, a->h_q, a->h_kv, a->indices ? a->topk : 0, pl);
   if (st != MLA_OK) return st;
   if (a->d_v != kDv) return MLA_ERR_UNSUPPORTED;
-  if ((a->indices != nullptr) != (a->is_fp8 != 0)) return MLA_ERR_UNSUPPORTED;  // dense fp8 / bf16 sparse
+  if (a->indices != nullptr && !a->is_fp8) return MLA_ERR_UNSUPPORTED;  // bf16 sparse
   if (a->indices != nullptr && a->topk < 1) return MLA_ERR_INVALID_ARG;
   if (!a->q || !a->k_cache || !a->block_table || !a->cache_seqlens || !a->tile_md || !a->num_splits || !a->out ||
       !a->lse || !a->err_word || !a->workspace)

@@ -95,8 +95,10 @@ def test_decode_rejects_bad_arguments_before_launch(lib):
     assert L.mla_decode(ctypes.byref(a), None) == _abi.MLA_ERR_UNSUPPORTED
     a.h_kv, a.d_v = 1, 256
     assert L.mla_decode(ctypes.byref(a), None) == _abi.MLA_ERR_UNSUPPORTED
-    a.d_v, a.is_fp8 = 512, 1                                                # fp8 without indices
+    a.d_v, a.is_fp8 = 512, 0
+    a.indices, a.topk = 1 << 20, 64                                         # sparse indices, bf16 cache
     assert L.mla_decode(ctypes.byref(a), None) == _abi.MLA_ERR_UNSUPPORTED
+    a.indices, a.topk = None, 0
     assert L.mla_get_metadata(None, 2, 1, 16, 1, 0, 4, None, None, None) == _abi.MLA_ERR_INVALID_ARG
     assert L.mla_get_metadata(None, 2, 1, 16, 3, 0, 4, None, None, None) == _abi.MLA_ERR_UNSUPPORTED
 

@@ -35,6 +35,15 @@ def test_row_tilings(h_q, s_q):
     assert_close(out, lse, *oracle(w))
 
 
+@pytest.mark.parametrize("h_q,s_q", [(128, 3), (128, 4), (64, 3), (64, 4)])
+def test_mtp_decode_more_tokens(h_q, s_q):
+    # s_q in {3, 4} new tokens (causal, bottom-right aligned) and 64-head tiles
+    w = I.make_workload("mtp", 3, s_q, h_q, [1000, 130, 2], causal=True, seed=7 * h_q + s_q)
+    out, lse, err = run(w)
+    assert err == 0
+    assert_close(out, lse, *oracle(w))
+
+
 def test_membound_small():
     w = I.make_config(2, batch=8, seqlen=1000)
     out, lse, err = run(w)
