@@ -13,6 +13,8 @@ mla_oracle    softmax(q K^T * scale) V and the log-sum-exp, walking the
               block_table; dense and sparse (top-k indices) key sets.
 brute         the same definition as pure-Python loops, for tiny inputs.
 metadata_ref  the split-KV scheduling plan, restated sequentially.
+fp8_writer_ref  quantisation of new key rows into the FP8 cache row format
+              (per-128 scale = max|x| / 448, e4m3 round-to-nearest-even).
 
 Parity pins: every function here is pinned by ``tests/test_oracle_*.py``
 against brute force, closed forms and invariants (no function is unpinned).
