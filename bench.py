@@ -171,6 +171,47 @@ def cpu_oracle_sample(w, budget_s: float):
     return kv_bytes / el / 1e9, flops / el / 1e12, desc, _blas_threads()
 
 
+def bench_fp8_writer(args) -> int:
+    """The FP8 cache writer on one GPU: 2 Mi new key rows (2.3 GB of bf16)
+    quantised into a 1.3 GB FP8 cache at shuffled slots.  A row moves 1152 B
+    in, 656 B out and a 4-B slot; the inputs exceed L2, so nothing is flushed.
+    One JSON line: GB/s against the measured copy bandwidth."""
+    import torch
+    import mla_decode_attention_get_b200 as M
+    hbm = load_peaks()[0]
+    n = 2 << 20
+    g = torch.Generator(device="cuda").manual_seed(2024)
+    k = torch.randn((n, 576), generator=g, device="cuda", dtype=torch.float32).to(torch.bfloat16)
+    slots = torch.randperm(n, generator=g, device="cuda").to(torch.int32)
+    cache = torch.zeros((n // 64, 64, 1, 656), dtype=torch.uint8, device="cuda")
+    err = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    for _ in range(args.warmup):
+        M.fp8_cache_write(k, slots, cache, err)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    sampler = ClockSampler(torch.cuda.current_device(), None)
+    with sampler:
+        ev[0].record()
+        for _ in range(args.steps):
+            M.fp8_cache_write(k, slots, cache, err)
+        ev[1].record()
+        torch.cuda.synchronize()
+    ms = ev[0].elapsed_time(ev[1]) / args.steps
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())}")
+    moved = n * (1152 + 656 + 4)
+    gbs = moved / (ms * 1e-3) / 1e9
+    print(json.dumps({
+        "metric": "FP8 cache writer GB/s (bytes moved per row: 1152 in, 656 + 4 out)", "value": round(gbs, 1),
+        "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "dtype": "bf16->e4m3", "data": "synthetic",
+        "config": {"workload": "fp8 cache write n=2097152 rows, shuffled slots", "rows": n},
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(gbs / hbm, 4), "kernel": "fp8_cache_write_kernel", "kernel_ms": round(ms, 5)},
+        "gpu_launches": args.steps, "clocks": sampler.summary()}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -180,8 +221,12 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default="decode", choices=["decode", "fp8_cache_write"],
+                    help="decode (the step: scheduler + attention + combine) or the FP8 cache writer alone")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
+    if args.op == "fp8_cache_write":
+        return bench_fp8_writer(args)
 
     world = _env_int("WORLD_SIZE", 1)
     rank = _env_int("RANK", 0)

@@ -183,6 +183,34 @@ MLA_API int mla_decode_combine(const mla_decode_args* args, void* stream);
 MLA_API int mla_decode_noalloc(const mla_decode_args* args, void* stream);
 
 /* Human-readable name of a status code (static string). */
+/*
+ * FP8 cache writer: quantise n new key rows into the FP8 cache row format
+ * (FlashMLA walkthrough (sao.pub), section "二、核心功能与架构": 512 e4m3
+ * NoPE values + 4 float32 scales, one per 128 values + 64 bf16 RoPE values =
+ * 656 bytes) and store row i at slot_mapping[i] = page * 64 + row.  The pages
+ * fix the format; the scales follow the plainest reading: scale = max|x| / 448
+ * per 128-value group (float32), code = e4m3 round-to-nearest-even of
+ * x / scale (IEEE float32 division), saturating; an all-zero group gets scale
+ * 0 and codes 0; RoPE is copied.  (The decode reads these rows back with
+ * is_fp8.)
+ *
+ *   k_new         bf16 [n, 576] (device), rows k_row_stride elements apart
+ *                 (multiple of 8, >= 576), 16-B aligned; values finite
+ *   slot_mapping  int32 [n] (device); -1 skips a row; a slot outside
+ *                 [0, num_blocks * 64) is skipped and sets MLA_DEVERR_BLOCK_TABLE
+ *   kv_cache      uint8 [num_blocks, 64, 1, 656] (device, written), pages
+ *                 k_block_stride bytes apart (multiple of 16, >= 64 * 656),
+ *                 16-B aligned
+ *   err_word      int32 (device), caller-zeroed
+ * Asynchronous on `stream`; n == 0 launches nothing.  Two rows mapped to the
+ * same slot race.  Returns MLA_OK, MLA_ERR_INVALID_ARG or MLA_ERR_CUDA.
+ * (No counterpart call on the pages: it is the step that produces the cache
+ * the FP8 decode reads.)
+ */
+MLA_API int mla_fp8_cache_write(const void* k_new, int64_t k_row_stride, int32_t n, const int32_t* slot_mapping,
+                                void* kv_cache, int64_t k_block_stride, int32_t num_blocks, int32_t* err_word,
+                                void* stream);
+
 MLA_API const char* mla_status_string(int status);
 
 #ifdef __cplusplus

@@ -27,7 +27,7 @@ from ._abi import MlaError, D_QK, D_V, PAGE_SIZE, FP8_ROW_BYTES
 
 __all__ = ["get_mla_metadata", "flash_mla_with_kvcache", "MlaError", "mla_get_metadata", "mla_decode",
            "mla_decode_attention", "mla_decode_combine", "mla_decode_noalloc", "mla_metadata_shape",
-           "mla_workspace_bytes", "DecodeCall"]
+           "mla_workspace_bytes", "DecodeCall", "fp8_cache_write"]
 
 
 def _stream_ptr(device) -> int:
@@ -216,3 +216,34 @@ def flash_mla_with_kvcache(q: torch.Tensor, k_cache: torch.Tensor, block_table: 
         if e:
             raise MlaError(_abi.MLA_ERR_INVALID_ARG, f"device error word 0x{e:x}")
     return out, lse
+
+
+def fp8_cache_write(k_new: torch.Tensor, slot_mapping: torch.Tensor, kv_cache: torch.Tensor,
+                    err: Optional[torch.Tensor] = None, check: bool = False) -> torch.Tensor:
+    """Quantise new key rows into the FP8 cache (C ABI ``mla_fp8_cache_write``).
+
+    ``k_new`` bf16 [n, 576] on CUDA (rows contiguous); ``slot_mapping`` int32
+    [n] (page * 64 + row; -1 skips a row); ``kv_cache`` uint8
+    [num_blocks, 64, 1, 656], written in place.  Returns the int32 error word
+    (``err`` if given); with ``check=True`` it synchronises and raises if a
+    slot was out of range."""
+    _require(k_new.is_cuda and k_new.dtype == torch.bfloat16 and k_new.dim() == 2 and k_new.shape[1] == D_QK
+             and k_new.stride(1) == 1, "k_new must be bf16 [n, 576] with contiguous rows")
+    _require(slot_mapping.dtype == torch.int32 and slot_mapping.is_contiguous()
+             and slot_mapping.shape == (k_new.shape[0],), "slot_mapping must be contiguous int32 [n]")
+    if kv_cache.dtype != torch.uint8:
+        kv_cache = kv_cache.view(torch.uint8)
+    _require(kv_cache.dim() == 4 and kv_cache.shape[1] == PAGE_SIZE and kv_cache.shape[2] == 1
+             and kv_cache.shape[3] == FP8_ROW_BYTES and kv_cache[0].is_contiguous(),
+             "kv_cache must be uint8 [num_blocks, 64, 1, 656] with contiguous pages")
+    if err is None:
+        err = torch.zeros((1,), dtype=torch.int32, device=k_new.device)
+    st = _abi.lib().mla_fp8_cache_write(k_new.data_ptr(), k_new.stride(0), k_new.shape[0], slot_mapping.data_ptr(),
+                                        kv_cache.data_ptr(), kv_cache.stride(0), kv_cache.shape[0], err.data_ptr(),
+                                        torch.cuda.current_stream(k_new.device).cuda_stream)
+    _abi.check(st, "mla_fp8_cache_write")
+    if check:
+        torch.cuda.synchronize(k_new.device)
+        if int(err.item()) != 0:
+            raise RuntimeError(f"fp8_cache_write: device error word {int(err.item())}")
+    return err

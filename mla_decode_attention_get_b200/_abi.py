@@ -30,7 +30,8 @@ FP8_ROW_BYTES = 656
 
 # Every symbol include/mla_decode.h declares.
 EXPORTS = ("mla_metadata_shape", "mla_get_metadata", "mla_workspace_bytes", "mla_decode",
-           "mla_decode_attention", "mla_decode_combine", "mla_decode_noalloc", "mla_status_string")
+           "mla_decode_attention", "mla_decode_combine", "mla_decode_noalloc", "mla_fp8_cache_write",
+           "mla_status_string")
 
 # Size of the scratch array built into the library for mla_decode_noalloc.
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -91,6 +92,7 @@ def lib() -> ctypes.CDLL:
         L.mla_workspace_bytes.argtypes = [i, i, i, i, i, p(ctypes.c_size_t)]
         for name in ("mla_decode", "mla_decode_attention", "mla_decode_combine", "mla_decode_noalloc"):
             getattr(L, name).argtypes = [p(DecodeArgs), v]
+        L.mla_fp8_cache_write.argtypes = [v, ctypes.c_int64, i, v, v, ctypes.c_int64, i, v, v]
         L.mla_status_string.argtypes = [i]
         L.mla_status_string.restype = ctypes.c_char_p
         for name in EXPORTS[:-1]:

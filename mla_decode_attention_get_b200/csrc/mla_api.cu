@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <cstdint>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -239,6 +240,23 @@ int mla_decode(const mla_decode_args* a, void* stream) {
   const int st = mla_decode_attention(a, stream);
   if (st != MLA_OK) return st;
   return mla_decode_combine(a, stream);
+}
+
+int mla_fp8_cache_write(const void* k_new, int64_t k_row_stride, int32_t n, const int32_t* slot_mapping,
+                        void* kv_cache, int64_t k_block_stride, int32_t num_blocks, int32_t* err_word,
+                        void* stream) {
+  if (n < 0 || num_blocks < 1) return MLA_ERR_INVALID_ARG;
+  if (n == 0) return MLA_OK;
+  if (!k_new || !slot_mapping || !kv_cache || !err_word) return MLA_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(kv_cache, 16) || !aligned(slot_mapping, 4) || !aligned(err_word, 4))
+    return MLA_ERR_INVALID_ARG;
+  if (k_row_stride < kDqk || k_row_stride % 8 != 0) return MLA_ERR_INVALID_ARG;
+  if (k_block_stride < int64_t(kPage) * mla::kFp8Row || k_block_stride % 16 != 0) return MLA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(num_blocks) * kPage > INT32_MAX) return MLA_ERR_INVALID_ARG;
+  const cudaError_t e = mla::launch_fp8_cache_write(static_cast<const uint16_t*>(k_new), k_row_stride, n, slot_mapping,
+                                                    static_cast<uint8_t*>(kv_cache), k_block_stride, num_blocks,
+                                                    err_word, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 const char* mla_status_string(int status) {

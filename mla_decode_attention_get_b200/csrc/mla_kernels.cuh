@@ -98,4 +98,8 @@ int pair_cluster_capacity();
 
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream);
 
+cudaError_t launch_fp8_cache_write(const uint16_t* k_new, int64_t row_stride, int n, const int* slot_mapping,
+                                   uint8_t* cache, int64_t block_stride, int num_blocks, int* err,
+                                   cudaStream_t stream);
+
 }  // namespace mla

@@ -133,3 +133,22 @@ def test_decode_checks_alignment_and_workspace(lib):
     a.k_block_stride = 64 * 576 * 2
     a.q_batch_stride = 16 * 576 - 8
     assert L.mla_decode(ctypes.byref(a), None) == _abi.MLA_ERR_INVALID_ARG
+
+
+def test_fp8_cache_write_validates_before_launch(lib):
+    L = _abi.lib()
+    fake = 1 << 20
+    ok = dict(k=fake, rs=576, n=4, slots=fake, cache=fake, bs=64 * 656, nb=8, err=fake)
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return L.mla_fp8_cache_write(a["k"], a["rs"], a["n"], a["slots"], a["cache"], a["bs"], a["nb"], a["err"], None)
+
+    assert call(n=0) == _abi.MLA_OK                       # nothing to do: no launch
+    assert call(n=-1) == _abi.MLA_ERR_INVALID_ARG
+    assert call(k=0) == _abi.MLA_ERR_INVALID_ARG
+    assert call(k=fake + 8) == _abi.MLA_ERR_INVALID_ARG   # not 16-B aligned
+    assert call(rs=572) == _abi.MLA_ERR_INVALID_ARG       # rows overlap
+    assert call(rs=580) == _abi.MLA_ERR_INVALID_ARG       # row starts not 16-B aligned
+    assert call(bs=64 * 656 - 16) == _abi.MLA_ERR_INVALID_ARG
+    assert call(nb=0) == _abi.MLA_ERR_INVALID_ARG
