@@ -212,6 +212,49 @@ def bench_fp8_writer(args) -> int:
     return 0
 
 
+def bench_sparse_prefill(args) -> int:
+    """A prefill-shaped sparse call on one GPU: 2 sequences of 32768 cached
+    FP8 tokens, 1024 new query tokens each, h_q = 128, a top-k of 2048
+    positions per token (the same kernels as the sparse decode: one
+    scheduler unit per token).  One JSON line: TFLOP/s against the measured
+    sustained bf16 GEMM rate."""
+    import torch
+    import mla_decode_attention_get_b200 as M
+    from mla_decode_attention_get_b200 import inputs as I
+    _, tc, tc_sus, _ = load_peaks()
+    w = I.make_workload("sparse prefill b=2 s_q=1024 h_q=128 L=32768 topk=2048", 2, 1024, 128, [32768, 32768],
+                        fp8=True, topk=2048, seed=3001)
+    flops, kv_bytes = I.flops_and_bytes(w)
+    t = I.to_device(w)
+    md, ns = M.get_mla_metadata(t["sl"], w.s_q * w.h_q, 1, s_q=w.s_q, topk=w.topk)
+    call = M.prepare_decode(t["q"], t["kv"], t["bt"], t["sl"], 512, md, ns, w.softmax_scale, False, True, t["idx"])
+    for _ in range(args.warmup):
+        call.decode()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    sampler = ClockSampler(torch.cuda.current_device(), None)
+    with sampler:
+        ev[0].record()
+        for _ in range(args.steps):
+            call.decode()
+        ev[1].record()
+        torch.cuda.synchronize()
+    ms = ev[0].elapsed_time(ev[1]) / args.steps
+    if int(call._keep[9].item()) != 0:
+        raise RuntimeError(f"device error word {int(call._keep[9].item())}")
+    tfs = flops / (ms * 1e-3) / 1e12
+    print(json.dumps({
+        "metric": "sparse prefill TFLOP/s (2*(576+512) FLOPs per (row, valid index))", "value": round(tfs, 1),
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "dtype": "f16 (FP8 cache dequantised)", "data": "synthetic",
+        "config": {"workload": w.name, "flops": flops, "kv_bytes": kv_bytes},
+        "roofline": {"bound": "tensor", "achieved": round(tfs, 1), "peak": tc_sus, "unit": "TFLOP/s",
+                     "frac": round(tfs / tc_sus, 4), "peak_kind": "sustained bf16 GEMM",
+                     "frac_of_burst_peak": round(tfs / tc, 4)},
+        "gpu_launches": 3 * args.steps, "clocks": sampler.summary()}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -221,12 +264,15 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default="decode", choices=["decode", "fp8_cache_write"],
-                    help="decode (the step: scheduler + attention + combine) or the FP8 cache writer alone")
+    ap.add_argument("--op", default="decode", choices=["decode", "fp8_cache_write", "sparse_prefill"],
+                    help="decode (the step: scheduler + attention + combine), the FP8 cache writer alone, "
+                         "or a prefill-shaped sparse call")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
     if args.op == "fp8_cache_write":
         return bench_fp8_writer(args)
+    if args.op == "sparse_prefill":
+        return bench_sparse_prefill(args)
 
     world = _env_int("WORLD_SIZE", 1)
     rank = _env_int("RANK", 0)

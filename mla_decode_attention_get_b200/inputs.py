@@ -241,8 +241,8 @@ def make_config(cfg: int, *, batch: Optional[int] = None, seqlen: Optional[int] 
 def flops_and_bytes(w: Workload):
     """Algorithmic work of one decode call: 2*(576+512) FLOPs per unmasked
     (query row, key) pair, and 1152 B per visible bf16 cache row or 656 B per
-    valid fp8 index (each row counted once per sequence, or per query token on
-    the sparse path)."""
+    fp8 row (each row counted once per sequence on the dense paths, or once
+    per valid index of a query token on the sparse path)."""
     pairs = 0
     if w.indices is not None:
         pairs = int((w.indices >= 0).sum()) * w.h_q
@@ -252,7 +252,7 @@ def flops_and_bytes(w: Workload):
             for i in range(w.s_q):
                 vis = L if not w.causal else max(0, min(L, L - w.s_q + i + 1))
                 pairs += vis * w.h_q
-        kv_bytes = int(w.cache_seqlens.astype(np.int64).sum()) * D_QK * 2
+        kv_bytes = int(w.cache_seqlens.astype(np.int64).sum()) * (FP8_ROW_BYTES if w.fp8 else D_QK * 2)
     return 2 * (D_QK + D_V) * pairs, kv_bytes
 
 

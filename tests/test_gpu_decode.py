@@ -80,6 +80,16 @@ def test_output_independent_of_partition_count(parts):
     assert_close(out, lse, *oracle(w))
 
 
+def test_sparse_prefill_shape():
+    # prefill-shaped sparse call: many query tokens, each with its own top-k
+    # (one scheduler unit per token)
+    w = I.make_workload("sprefill", 1, 96, 64, [5000], fp8=True, topk=512, seed=51,
+                        pad_rows_per_token=32, num_padded_rows=10)
+    out, lse, err = run(w)
+    assert err == 0
+    assert_close(out, lse, *oracle(w))
+
+
 @pytest.mark.parametrize("parts", [1, 3, 148])
 def test_sparse_output_independent_of_partition_count(parts):
     w = I.make_workload("sp", 3, 2, 32, [4000, 700, 90], fp8=True, topk=300, seed=5,
