@@ -84,6 +84,7 @@ constexpr int kRows = 64;                     // query rows per CTA = M of every
 constexpr int kStages = 3;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemQCol = 128;           // Q tile columns 128..415 in lanes 16-31
+constexpr int kPChunk = kChunks - 1;          // the RoPE chunk of a stage, reused for the page's P tile
 
 constexpr int kWarpLoad = 0, kWarpMma = 1, kWarpSoftmax0 = 2, kWarpDequant0 = 6;
 constexpr int kDequantWarps = 8;              // FP8 path: warp dq converts keys [8 dq, 8 dq + 8)
@@ -91,16 +92,18 @@ constexpr int kThreadsDense = 32 * kWarpDequant0;
 constexpr int kThreadsFp8 = 32 * (kWarpDequant0 + kDequantWarps);
 
 struct Smem {
-  static constexpr int kv_off = 0;                               // page ring
-  static constexpr int p_off = kv_off + kStages * kPageBytes;    // P tile: [64 rows x 64 keys] bf16
-  static constexpr int bar_off = p_off + kRows * 128;
-  // kv_full[S], kv_empty[S], s_full[2], s_empty[2], q_full, p_full, p_empty, done
-  static constexpr int n_bars = 2 * kStages + 4 + 4;
+  // page ring; once QK of a page has completed, the page's RoPE chunk holds
+  // its P tile ([64 rows x 64 keys], the same 128-B swizzled geometry)
+  static constexpr int kv_off = 0;
+  static constexpr int bar_off = kv_off + kStages * kPageBytes;
+  // kv_full[S], kv_empty[S], s_full[2], s_empty[2], q_full, p_full[S], done
+  static constexpr int n_bars = 3 * kStages + 6;
   static constexpr int info_off = bar_off + n_bars * 8;
   static constexpr int info_bytes = kStages * 16;                // per stage: int nvalid; uint16 mask[4]
   static constexpr int misc_off = info_off + info_bytes;         // tmem base, abort flag
   static constexpr int total = misc_off + 16;
-  static_assert(kv_off % 1024 == 0 && p_off % 1024 == 0, "tiles must stay 1024-B aligned");
+  static_assert(kv_off % 1024 == 0 && kPageBytes % 1024 == 0 && kChunkBytes % 1024 == 0,
+                "tiles must stay 1024-B aligned");
   static_assert(total <= 232448, "shared memory budget");
 };
 
@@ -116,8 +119,7 @@ struct Bars {
   uint64_t* s_full;
   uint64_t* s_empty;
   uint64_t* q_full;
-  uint64_t* p_full;
-  uint64_t* p_empty;
+  uint64_t* p_full;     // per stage: P of the stage's page written (4 softmax warps)
   uint64_t* done;
 };
 
@@ -391,14 +393,11 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
   constexpr uint32_t idesc_qk = FP8 ? idesc_f16_f32(kRows, kPage, false, false) : idesc_bf16_f32(kRows, kPage, false, false);
   constexpr uint32_t idesc_pv = FP8 ? idesc_f16_f32(kRows, 256, false, true) : idesc_bf16_f32(kRows, 256, false, true);
   const uint32_t tmem_q = tmem_base + (16u << 16) + kTmemQCol;   // A operand of QK (lanes 16-31)
-  const uint64_t p_desc = sdesc_sw128(smem_u32(smem + Smem::p_off), 16, 1024);
-  uint64_t k_desc[kStages], v_desc[kStages];
-#pragma unroll
-  for (int s = 0; s < kStages; ++s) {
-    const uint32_t a = smem_u32(smem + Smem::kv_off + s * kPageBytes);
-    k_desc[s] = sdesc_sw128(a, 16, 1024);
-    v_desc[s] = sdesc_sw128(a, kChunkBytes, 1024);
-  }
+  // descriptors of stage 0; a stage's own add its offset to the 16-B address field
+  const uint32_t ring = smem_u32(smem + Smem::kv_off);
+  const uint64_t k_desc0 = sdesc_sw128(ring, 16, 1024);
+  const uint64_t v_desc0 = sdesc_sw128(ring, kChunkBytes, 1024);
+  const uint64_t p_desc0 = sdesc_sw128(ring + kPChunk * kChunkBytes, 16, 1024);
   const uint32_t tmem_s0 = tmem_base + (16u << 16);    // S buffers: lanes 16-31 of each quadrant
 
   Cursor qk = cursor_begin(p, part);
@@ -419,25 +418,26 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
   while (pv.valid) {
     bool progressed = false;
     // PV(pv.t): after QK(pv.t) was issued and the softmax wrote P(pv.t)
-    if (pv.t < qk.t && ready(bars.p_full, pv.t & 1)) {
+    if (pv.t < qk.t && ready(&bars.p_full[pv.t % kStages], (pv.t / kStages) & 1)) {
       if (lane == 0) MLA_TRACE_EV(3, pv.t);
       tc_fence_after();
       const int s = pv.t % kStages;
       if (qk_nv[s] > 0) {
         const bool acc0 = (o_seg == pv.seg);
-        const uint64_t vd = v_desc[s];
+        const uint64_t vd = v_desc0 + ((s * kPageBytes) >> 4);
+        const uint64_t pd = p_desc0 + ((s * kPageBytes) >> 4);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            umma_bf16_elect(tmem_base + h * 256, p_desc + ((k * 32) >> 4),
+            umma_bf16_elect(tmem_base + h * 256, pd + ((k * 32) >> 4),
                             vd + ((4 * h * kChunkBytes + k * 2048) >> 4), idesc_pv, (acc0 || k > 0) ? 1u : 0u);
           }
         }
         o_seg = pv.seg;
       }
+      // the stage (K, V and P of the page) is free once PV has completed
       umma_commit_elect(&bars.kv_empty[s]);
-      umma_commit_elect(bars.p_empty);
       if (lane == 0) MLA_TRACE_EV(14, pv.t);
       cursor_next(p, part, pv);
       progressed = true;
@@ -454,7 +454,7 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
         const int nv = stage_nvalid(info[s], FP8);
         qk_nv[s] = nv;
         if (nv > 0) {
-          const uint64_t kd = k_desc[s];
+          const uint64_t kd = k_desc0 + ((s * kPageBytes) >> 4);
           const uint32_t d = tmem_s0 + sb * kPage;
 #pragma unroll
           for (int c = 0; c < kChunks; ++c) {
@@ -544,6 +544,9 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
   const int R = p.rows_per_unit;
   const int grow = blockIdx.y * kRows + r;           // row within the unit
   const bool row_valid = grow < R;
+  // A warp whose 16 rows are all padding keeps the barrier protocol but does
+  // no math: the O rows its P rows feed are never read.
+  const bool warp_live = static_cast<int>(blockIdx.y) * kRows + 16 * q4 < R;
   const float scale_log2 = p.scale_log2;
   const int h_q = p.h_q, s_q = p.s_q;
   const int tok_dense = grow / h_q;                  // dense path: the row's query token
@@ -551,7 +554,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
   const bool causal = !sparse && p.causal != 0;
   const uint32_t s_taddr = tmem_base + (static_cast<uint32_t>(32 * q4 + 16) << 16);
   const uint32_t o_taddr = tmem_base + (static_cast<uint32_t>(32 * q4) << 16);
-  const uint32_t p_row = smem_u32(smem + Smem::p_off) + r * 128;
+  const uint32_t p_row0 = smem_u32(smem + Smem::kv_off + kPChunk * kChunkBytes) + r * 128;
   const int key0 = 32 * half;                        // first key (and dim offset) of this thread's half
   const uint32_t tq_lane = tmem_base + (static_cast<uint32_t>(32 * q4 + 16) << 16) + kTmemQCol;
 
@@ -588,14 +591,15 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
       if (lane == 0 && q4 == 2) MLA_TRACE_EV(4, t);
       tc_fence_after();
       const int nv = stage_nvalid(info[s], FP8);
+      const bool work = nv > 0 && warp_live;
       float x[32];
-      if (nv > 0) tmem_ld_16x32bx2_x32(s_taddr + sb * kPage, x);
+      if (work) tmem_ld_16x32bx2_x32(s_taddr + sb * kPage, x);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.s_empty[sb]);
 
       float tmax = -INFINITY;
-      if (nv > 0) {
+      if (work) {
         uint32_t vmask;
         if (FP8) {
           vmask = static_cast<uint32_t>(info[s].mask[2 * half]) |
@@ -618,15 +622,18 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
       const bool need = tmax > m_run + kRescaleThreshold;
       if (lane == 0 && q4 == 2) MLA_TRACE_EV(11, t);
 
-      if (t > 0 && !mbar_wait(bars.p_empty, (t - 1) & 1, abort_flag)) { ok = false; return false; }
       if (lane == 0 && q4 == 2) MLA_TRACE_EV(6, t);
-      tc_fence_after();
       if (__any_sync(0xffffffffu, need)) {
         const float m_new = need ? fmaxf(m_run, tmax) : m_run;
         const float alpha = (m_new == m_run) ? 1.f : fast_exp2(m_run - m_new);   // m_run = -inf -> 0
         l_run *= alpha;
         m_run = m_new;
         if (__any_sync(0xffffffffu, any_pv && alpha != 1.f)) {
+          // O holds every PV of the segment once PV(t-1), which frees its
+          // stage, has completed (any_pv implies t > 0)
+          const int tp = t - 1;
+          if (!mbar_wait(&bars.kv_empty[tp % kStages], (tp / kStages) & 1, abort_flag)) { ok = false; return false; }
+          tc_fence_after();
           if (lane == 0 && q4 == 2) MLA_TRACE_EV(9, t);
 #pragma unroll 1
           for (int c0 = 0; c0 < kDv; c0 += 64) {
@@ -639,11 +646,13 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
         }
       }
 
-      // P = exp2(s - m) as bf16: this thread's 64-B half of row r of the
-      // K-major swizzled P tile
+      // P = exp2(s - m) as bf16 (f16 for FP8): this thread's 64-B half of
+      // row r of the K-major swizzled P tile in the page's RoPE chunk, whose
+      // last reader, QK of this page, has completed
       const float m_safe = m_run == -INFINITY ? 0.f : m_run;
+      const uint32_t p_row = p_row0 + s * kPageBytes;
       uint32_t pk[16];
-      if (nv > 0) {
+      if (work) {
         float lsum = 0.f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -657,11 +666,13 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
 #pragma unroll
         for (int i = 0; i < 16; ++i) pk[i] = 0u;
       }
+      if (warp_live) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int chunk = 4 * half + c;
-        st_shared_v4(p_row + ((chunk ^ (r & 7)) << 4),
-                     make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]));
+        for (int c = 0; c < 4; ++c) {
+          const int chunk = 4 * half + c;
+          st_shared_v4(p_row + ((chunk ^ (r & 7)) << 4),
+                       make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]));
+        }
       }
       if (lane == 0 && q4 == 2) MLA_TRACE_EV(13, t);
 
@@ -680,14 +691,14 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bars.p_full);
+      if (lane == 0) mbar_arrive(&bars.p_full[s]);
       if (lane == 0 && q4 == 2) MLA_TRACE_EV(7, t);
       if (nv > 0) any_pv = true;
 
-      if (j == je - 1) {
-        stage_next_q(u + 1);
+      if (j == je - 1) stage_next_q(u + 1);
+      if (j == je - 1 && warp_live) {
         // ------------------------------------------------ epilogue of the segment
-        if (!mbar_wait(bars.p_empty, t & 1, abort_flag)) { ok = false; return false; }
+        if (!mbar_wait(&bars.kv_empty[s], (t / kStages) & 1, abort_flag)) { ok = false; return false; }   // PV(t) done
         tc_fence_after();
         const float l = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
         const bool has = any_pv && l > 0.f;
@@ -758,8 +769,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreadsDense, 1)
   bars.s_empty = bar + 2 * kStages + 2;
   bars.q_full = bar + 2 * kStages + 4;
   bars.p_full = bar + 2 * kStages + 5;
-  bars.p_empty = bar + 2 * kStages + 6;
-  bars.done = bar + 2 * kStages + 7;
+  bars.done = bar + 3 * kStages + 5;
   StageInfo* info = reinterpret_cast<StageInfo*>(smem + Smem::info_off);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::misc_off + 4);
@@ -770,6 +780,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreadsDense, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars.kv_full[s], FP8 ? kDequantWarps : 1);
       mbar_init(&bars.kv_empty[s], 1);
+      mbar_init(&bars.p_full[s], 4);
       info[s].nvalid = 0;
       for (int w = 0; w < 4; ++w) info[s].mask[w] = 0;
     }
@@ -778,8 +789,6 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreadsDense, 1)
       mbar_init(&bars.s_empty[i], 4);
     }
     mbar_init(bars.q_full, 4);
-    mbar_init(bars.p_full, 4);
-    mbar_init(bars.p_empty, 1);
     mbar_init(bars.done, 1);
     fence_barrier_init();
   }
