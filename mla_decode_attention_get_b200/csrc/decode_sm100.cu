@@ -279,24 +279,32 @@ __device__ __forceinline__ void dequant_role(const DecodeParams& p, const Partit
     return v;
   };
 
+  // Pipeline over tiles: while tile t converts, the rows of tile t+1 are
+  // warmed in L2, the table entry of tile t+2 and the index of tile t+3 are
+  // in flight.
   Cursor cur = cursor_begin(p, part);
   Cursor nxt = cur;
   cursor_next(p, part, nxt);
+  Cursor nxt2 = nxt;
+  cursor_next(p, part, nxt2);
   int pos_c = fetch_pos(cur);
   int phys_c = -1;
   bool valid_c = finish_resolve(cur, start_resolve(cur, pos_c), phys_c);
   int pos_n = fetch_pos(nxt);
+  Pending pend_n = start_resolve(nxt, pos_n);
+  int pos_nn = fetch_pos(nxt2);
   int t = 0;
   while (cur.valid) {
     const int s = t % kStages;
+    int phys_n = -1;
+    const bool valid_n = finish_resolve(nxt, pend_n, phys_n);
+    if (valid_n && lane < 8) bulk_prefetch_l2(row_ptr(phys_n, pos_n), kFp8Row);
+    const Pending pend_nn = start_resolve(nxt2, pos_nn);
+    Cursor nxt3 = nxt2;
+    cursor_next(p, part, nxt3);
+    const int pos_nnn = fetch_pos(nxt3);
     if (!mbar_wait(&bars.kv_empty[s], ((t / kStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
     if (lane == 0 && dq == 0) MLA_TRACE_EV(0, t);
-    Cursor nxt2 = nxt;
-    cursor_next(p, part, nxt2);
-    const int pos_nn = fetch_pos(nxt2);            // tile t+2: in flight for a whole tile
-    const Pending pend = start_resolve(nxt, pos_n);  // tile t+1: in flight while this tile converts
-    int phys_n = -1;
-    bool valid_n = false;
     uint8_t* stage = smem + Smem::kv_off + s * kPageBytes;
     {
       uint2 n0[8], n1[8], rp[8];
@@ -353,9 +361,6 @@ __device__ __forceinline__ void dequant_role(const DecodeParams& p, const Partit
         }
       }
     }
-    // tile t+1 resolved: warm its rows in L2
-    valid_n = finish_resolve(nxt, pend, phys_n);
-    if (valid_n && lane < 8) bulk_prefetch_l2(row_ptr(phys_n, pos_n), kFp8Row);
     const uint32_t mask = __ballot_sync(0xffffffffu, valid_c) & 0xFFu;
     if (lane == 0) reinterpret_cast<uint8_t*>(info[s].mask)[dq] = static_cast<uint8_t>(mask);
     fence_proxy_async_smem();
@@ -364,10 +369,13 @@ __device__ __forceinline__ void dequant_role(const DecodeParams& p, const Partit
     if (lane == 0 && dq == 0) MLA_TRACE_EV(15, t);
     cur = nxt;
     nxt = nxt2;
+    nxt2 = nxt3;
     pos_c = pos_n;
     phys_c = phys_n;
     valid_c = valid_n;
     pos_n = pos_nn;
+    pend_n = pend_nn;
+    pos_nn = pos_nnn;
     ++t;
   }
   if (!ok && lane == 0) raise_abort(abort_flag, p.err);
