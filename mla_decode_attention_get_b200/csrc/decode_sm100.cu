@@ -298,7 +298,15 @@ __device__ __forceinline__ void dequant_role(const DecodeParams& p, const Partit
     const int s = t % kStages;
     int phys_n = -1;
     const bool valid_n = finish_resolve(nxt, pend_n, phys_n);
-    if (valid_n && lane < 8) bulk_prefetch_l2(row_ptr(phys_n, pos_n), kFp8Row);
+    if (valid_n) {
+      // the row of key (lane & 7) spans at most 7 lines; lane group lane >> 3
+      // warms lines g and g + 4 of it
+      const uintptr_t a = reinterpret_cast<uintptr_t>(row_ptr(phys_n, pos_n));
+      const uintptr_t first = a >> 7, last = (a + kFp8Row - 1) >> 7;
+      const uintptr_t g = static_cast<uintptr_t>(lane >> 3);
+      if (first + g <= last) prefetch_line_l2(reinterpret_cast<const void*>((first + g) << 7));
+      if (first + g + 4 <= last) prefetch_line_l2(reinterpret_cast<const void*>((first + g + 4) << 7));
+    }
     const Pending pend_nn = start_resolve(nxt2, pos_nn);
     Cursor nxt3 = nxt2;
     cursor_next(p, part, nxt3);

@@ -147,6 +147,11 @@ __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, i
 }
 
 // Warm L2 with `bytes` (multiple of 16) starting at a 16-B aligned address.
+// One 128-B line into L2 (fire and forget, through the load/store unit).
+__device__ __forceinline__ void prefetch_line_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
+
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
                : "memory");
