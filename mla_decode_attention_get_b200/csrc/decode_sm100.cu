@@ -245,23 +245,27 @@ __device__ __forceinline__ void dequant_role(const DecodeParams& p, const Partit
     if (!c.valid) return -1;
     const int pos_i = kPage * c.j + 8 * dq + kl;
     if (!sparse) return pos_i;
-    return pos_i < p.topk ? p.indices[static_cast<int64_t>(c.u) * p.topk + pos_i] : -1;
+    const bool in = pos_i < p.topk;
+    return ld_nc_s32_if(p.indices + (in ? static_cast<int64_t>(c.u) * p.topk + pos_i : 0), in, -1);
   };
   auto row_ptr = [&](int phys, int pos) -> const uint8_t* {
     return p.kv + static_cast<int64_t>(phys) * p.kv_block_stride + (pos & 63) * kFp8Row;
   };
 
-  // Loads behind resolving a tile: the length of its unit and the table entry
-  // of this lane's key, issued together (the entry speculatively).
+  // Loads behind resolving a tile: the length of its unit (as stored: a
+  // negative length admits no position) and the table entry of this lane's
+  // key, issued together (the entry speculatively) and first read a tile later.
   struct Pending {
     int pos, L, page_entry;
   };
   auto start_resolve = [&](const Cursor& c, int pos) -> Pending {
     Pending r{pos, 0, -1};
     if (!c.valid) return r;
-    const UnitInfo ui = unit_info(p, c.u);
-    r.L = ui.L;
-    if (pos >= 0) r.page_entry = page_of(p, ui.b, pos >> 6);
+    const int b = sparse ? c.u / p.s_q : c.u;
+    r.L = ld_nc_s32_if(p.seqlens + b, true, 0);
+    const int j = pos >> 6;
+    const bool in = pos >= 0 && j < p.bt_width;
+    r.page_entry = ld_nc_s32_if(p.block_table + (in ? static_cast<int64_t>(b) * p.bt_stride + j : 0), in, -1);
     return r;
   };
   auto finish_resolve = [&](const Cursor& c, const Pending& r, int& phys) -> bool {

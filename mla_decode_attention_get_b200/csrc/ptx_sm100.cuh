@@ -147,6 +147,20 @@ __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, i
 }
 
 // Warm L2 with `bytes` (multiple of 16) starting at a 16-B aligned address.
+// Read-only 32-bit load issued only when `pred` holds; otherwise `fallback`.
+// The result register is written by the load itself, so nothing waits on it
+// until it is first read (a select after a plain load would).
+__device__ __forceinline__ int ld_nc_s32_if(const int* ptr, bool pred, int fallback) {
+  int v = fallback;
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "setp.ne.b32 q, %2, 0;\n\t"
+      "@q ld.global.nc.b32 %0, [%1];\n\t}"
+      : "+r"(v)
+      : "l"(reinterpret_cast<uint64_t>(ptr)), "r"(pred ? 1 : 0));
+  return v;
+}
+
 // One 128-B line into L2 (fire and forget, through the load/store unit).
 __device__ __forceinline__ void prefetch_line_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
