@@ -39,7 +39,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # DRAM traffic (read + write bytes) of one attention-kernel launch per
 # workload, from one ncu capture of the current kernel (profiles/); None when
 # the kernel changed since or for workloads not captured.
-ATTN_TRAFFIC_BYTES = {2: 628_521_984, 3: 394_025_472, 5: 121_879_552}
+ATTN_TRAFFIC_BYTES = {2: 627_871_488, 3: 386_982_656, 5: 121_032_960}
 
 
 def _env_int(k, d):
