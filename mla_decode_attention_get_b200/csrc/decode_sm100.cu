@@ -20,6 +20,11 @@
 //    hold the two S buffers (columns 0-63, 64-127) and the query tile Q
 //    (columns 128-415, two bf16 per column), which QK reads straight from TMEM
 //    as its A operand.  With Q out of shared memory the page ring has 3 stages.
+//  * P of a page is written into the page's own RoPE box (64 rows x 128 B,
+//    the geometry of the swizzled P tile) once QK of the page has completed;
+//    PV of the page reads it before the stage is refilled.  So the softmax of
+//    the next page never waits for PV of this one: O is waited on only to
+//    rescale it and in a segment's epilogue.
 //  * Row r of the tile belongs to threads (r % 16) and (r % 16) + 16 of
 //    softmax warp r / 16: with 16-lane TMEM accesses each of the pair holds
 //    half of the row's 64 logits (and, in the epilogue, half of its O row), so
@@ -28,8 +33,9 @@
 //    = 9 boxes of 64 tokens x 64 dims) into the ring and warms L2 a few pages
 //    (and the next query tile) ahead; warp 1 issues the MMAs; warps 2-5 write
 //    each segment's query tile into TMEM, run the online softmax and the
-//    epilogue.  On the FP8 sparse path warps 6-13 gather the indexed rows and
-//    dequantise them into the same bf16 page layout.
+//    epilogue.  On the FP8 path warps 6-13 gather the indexed (or, dense,
+//    the paged) rows and dequantise them into the same page layout as f16;
+//    that path's MMAs run on f16 operands.
 //  * The running max only moves when a page's max exceeds it by more than
 //    2^8 (per row); the final division by the row sum uses the same stale
 //    max, so the result is exact.
