@@ -77,6 +77,22 @@ def test_output_independent_of_partition_count(parts):
     assert_close(out, lse, *oracle(w))
 
 
+def test_running_max_rescales():
+    # a few key rows on later pages get group scales 2^-5 (7-28 times the
+    # workload's): many rows' running max jumps by far more than the
+    # lazy-rescale threshold mid-sequence.  A power-of-two scale keeps every
+    # dequantised value exact in the kernel's f16 operands, so the big logits
+    # carry no dequantisation rounding.
+    w = I.make_workload("fp8dresc", 2, 1, 64, [3000, 2000], fp8=True, seed=47)
+    for b, L in enumerate(w.cache_seqlens):
+        for tok in (700 + b, 1500, int(L) - 3):
+            phys, row = w.block_table[b, tok // 64], tok % 64
+            w.kv_fp8[phys, row, 0, 512:528] = np.full(4, 2.0 ** -5, "<f4").view(np.uint8)
+    out, lse, err = run(w)
+    assert err == 0
+    assert_close(out, lse, *oracle(w))
+
+
 def test_larger_batch_sampled():
     rng = np.random.default_rng(46)
     L = rng.integers(1, 6000, size=32)
