@@ -8,6 +8,7 @@ import torch
 
 from mla_decode_attention_get_b200 import inputs as I
 from gpu_util import assert_close, oracle, run, upload
+import rescale_cases as RC
 
 pytestmark = pytest.mark.gpu
 
@@ -72,40 +73,18 @@ def test_fp8_sparse_small():
     assert_close(out, lse, *oracle(w))
 
 
-def _scale_bf16_row(w, phys, row, factor):
-    bits = w.kv_bits[phys, row, 0, :].astype(np.uint32) << 16
-    w.kv_bits[phys, row, 0, :] = I.f32_to_bf16_bits(bits.view(np.float32) * factor)
-
-
-def _boost_fp8_row(w, phys, row):
-    # all four group scales of the row (bytes 512..527, little-endian f32) set
-    # to 2^-5, 7-28 times the workload's scales: every dequantised value
-    # (an e4m3 value times a power of two) is then exact in the kernel's f16
-    # operands, so the big logits this makes carry no dequantisation rounding
-    w.kv_fp8[phys, row, 0, 512:528] = np.full(4, 2.0 ** -5, "<f4").view(np.uint8)
-
-
 @pytest.mark.parametrize("h_q,s_q,causal", [(16, 1, False), (128, 1, False), (64, 2, True)])
 def test_running_max_rescales(h_q, s_q, causal):
-    # a few key rows on later pages scaled x12: many rows' running max jumps by
-    # far more than the lazy-rescale threshold mid-sequence, while PV of the
-    # preceding pages may still be in flight
-    w = I.make_workload("rescale", 2, s_q, h_q, [3000, 2000], causal=causal, seed=50 + h_q)
-    for b, L in enumerate(w.cache_seqlens):
-        for tok in (700 + b, 1500, int(L) - 3):
-            _scale_bf16_row(w, w.block_table[b, tok // 64], tok % 64, 12.0)
+    # many rows' running max jumps far past the lazy-rescale threshold
+    # mid-sequence, while PV of the preceding pages may still be in flight
+    w = RC.bf16_case(h_q, s_q, causal)
     out, lse, err = run(w)
     assert err == 0
     assert_close(out, lse, *oracle(w))
 
 
 def test_running_max_rescales_fp8_sparse():
-    # the rows named at index slots 700 and 1500 of every token boosted
-    w = I.make_workload("rescale8", 2, 1, 128, [4000, 3000], fp8=True, topk=2048, seed=53)
-    for b in range(w.batch):
-        for slot in (700, 1500):
-            pos = int(w.indices[b, 0, slot])
-            _boost_fp8_row(w, w.block_table[b, pos // 64], pos % 64)
+    w = RC.fp8_sparse_case()
     out, lse, err = run(w)
     assert err == 0
     assert_close(out, lse, *oracle(w))

@@ -12,6 +12,7 @@ import pytest
 
 from mla_decode_attention_get_b200 import inputs as I
 from gpu_util import assert_close, oracle, run
+import rescale_cases as RC
 
 pytestmark = pytest.mark.gpu
 
@@ -78,16 +79,9 @@ def test_output_independent_of_partition_count(parts):
 
 
 def test_running_max_rescales():
-    # a few key rows on later pages get group scales 2^-5 (7-28 times the
-    # workload's): many rows' running max jumps by far more than the
-    # lazy-rescale threshold mid-sequence.  A power-of-two scale keeps every
-    # dequantised value exact in the kernel's f16 operands, so the big logits
-    # carry no dequantisation rounding.
-    w = I.make_workload("fp8dresc", 2, 1, 64, [3000, 2000], fp8=True, seed=47)
-    for b, L in enumerate(w.cache_seqlens):
-        for tok in (700 + b, 1500, int(L) - 3):
-            phys, row = w.block_table[b, tok // 64], tok % 64
-            w.kv_fp8[phys, row, 0, 512:528] = np.full(4, 2.0 ** -5, "<f4").view(np.uint8)
+    # many rows' running max jumps far past the lazy-rescale threshold
+    # mid-sequence (rows boosted with exact power-of-two scales)
+    w = RC.fp8_dense_case()
     out, lse, err = run(w)
     assert err == 0
     assert_close(out, lse, *oracle(w))
