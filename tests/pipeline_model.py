@@ -1,0 +1,322 @@
+"""A host-side model of the decode kernel's synchronisation protocol.
+
+Test infrastructure only.  It restates, role by role, the mbarrier hand-offs
+of one CTA of the decode kernel in `csrc/decode_sm100.cu`:
+- the page producer: the TMA warp on the bf16 path, or 8 gather warps on the
+  FP8 path;
+- the MMA warp's event loop;
+- the four softmax warps, with idle padding warps, lazy rescales, segment
+  epilogues and query-tile staging.
+A random scheduler then interleaves the roles, the landing of page loads and
+the in-order completion of the tensor pipe.
+
+An mbarrier is modelled by its count, its pending arrivals and the number of
+phases it has completed.  A wait on parity P passes when the completed count
+has the other parity, as the hardware does.  The model also knows which
+phase each wait and each arrival means, and flags:
+- a wait that passes on a different phase than the one it means (parity
+  aliasing);
+- an arrival that lands in another page's phase;
+- a data hazard: an MMA that reads a stage, S buffer, P tile or query tile
+  its producer has not finished, or a write to one that a reader still needs;
+  a rescale or epilogue read of O while PV may still update it;
+- a deadlock: nothing can move, and work is left.
+
+`mutation` switches on one planted protocol mistake, to show that the checks
+catch it:
+- "shared_p_full": one p_full barrier for all pages;
+- "no_rescale_wait": rescale O without waiting for PV of the previous page;
+- "single_pv_barrier": the epilogue waits for PV through one barrier
+  committed per page, with parity t & 1.
+"""
+from __future__ import annotations
+
+import random
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional
+
+STAGES = 3
+WARPS = 4            # softmax warps, one per TMEM lane quadrant
+GATHER_WARPS = 8     # FP8 path
+
+
+class ProtocolError(AssertionError):
+    pass
+
+
+class Barrier:
+    def __init__(self, name: str, count: int):
+        self.name, self.count, self.pending, self.completed = name, count, count, 0
+
+    def arrive(self, phase: int):
+        if phase != self.completed:
+            raise ProtocolError(f"{self.name}: arrival meant for phase {phase} lands in phase {self.completed}")
+        self.pending -= 1
+        if self.pending == 0:
+            self.completed += 1
+            self.pending = self.count
+
+    def passes(self, phase: int) -> bool:
+        """Hardware parity test of a wait that means "phase `phase` has
+        completed" (phase -1: the barrier's initial state)."""
+        ok = (self.completed & 1) != (phase & 1)
+        if ok and self.completed != phase + 1:
+            raise ProtocolError(f"{self.name}: wait for phase {phase} passes at {self.completed} completed phases")
+        return ok
+
+
+@dataclass
+class Plan:
+    segments: List[int]                 # pages per segment, in order
+    live_warps: int                     # softmax warps with at least one real row
+    fp8: bool = False
+    rescale: Optional[Dict] = None      # (warp, page) -> bool: a rescale is needed
+
+
+@dataclass
+class State:
+    stage_page: List[Optional[int]] = field(default_factory=lambda: [None] * STAGES)
+    stage_writers: List[int] = field(default_factory=lambda: [0] * STAGES)
+    qk_done: set = field(default_factory=set)
+    pv_done: set = field(default_factory=set)
+    p_written: Dict[int, int] = field(default_factory=dict)
+    s_reading: Dict[int, set] = field(default_factory=lambda: {0: set(), 1: set()})
+    s_page: Dict[int, Optional[int]] = field(default_factory=lambda: {0: None, 1: None})
+    o_busy: set = field(default_factory=set)
+    q_seg: int = -1                     # segment whose query tile is in TMEM
+    q_writes: Dict[int, int] = field(default_factory=dict)
+    epilogue_done: Dict[int, int] = field(default_factory=dict)
+
+
+class Model:
+    def __init__(self, plan: Plan, seed: int, mutation: Optional[str] = None):
+        self.plan, self.rng, self.mut = plan, random.Random(seed), mutation
+        self.T = sum(plan.segments)
+        self.seg_of, self.first_of_seg = [], set()
+        t = 0
+        for k, n in enumerate(plan.segments):
+            self.first_of_seg.add(t)
+            self.seg_of += [k] * n
+            t += n
+        S = STAGES
+        self.kv_full = [Barrier(f"kv_full[{s}]", GATHER_WARPS if plan.fp8 else 1) for s in range(S)]
+        self.kv_empty = [Barrier(f"kv_empty[{s}]", 1) for s in range(S)]
+        self.s_full = [Barrier(f"s_full[{b}]", 1) for b in range(2)]
+        self.s_empty = [Barrier(f"s_empty[{b}]", WARPS) for b in range(2)]
+        self.q_full = Barrier("q_full", WARPS)
+        if mutation == "shared_p_full":
+            shared = Barrier("p_full", WARPS)
+            self.p_full = [shared] * S
+        else:
+            self.p_full = [Barrier(f"p_full[{s}]", WARPS) for s in range(S)]
+        self.pv_bar = Barrier("pv_done", 1)          # only the planted mistake waits on it
+        self.st = State()
+        self.pipe: List[tuple] = []                  # tensor pipe, in order
+        self.loads: List[int] = []                   # pages in flight (bf16 path)
+
+    # -- phase bookkeeping ---------------------------------------------------
+    def p_full_phase(self, t):
+        return t if self.mut == "shared_p_full" else t // STAGES
+
+    # -- roles (generators yielding ("wait", pred) or ("step",)) -------------
+    def producer(self):
+        for t in range(self.T):
+            s = t % STAGES
+            yield ("wait", lambda s=s, t=t: self.kv_empty[s].passes(t // STAGES - 1))
+            self._stage_write_begin(s, t)
+            self.loads.append(t)
+            yield ("step",)
+
+    def gather(self, w):
+        for t in range(self.T):
+            s = t % STAGES
+            yield ("wait", lambda s=s, t=t: self.kv_empty[s].passes(t // STAGES - 1))
+            self._stage_write_begin(s, t)
+            yield ("step",)
+            self._stage_write_end(s, t)
+            self.kv_full[s].arrive(t // STAGES)
+            yield ("step",)
+
+    def mma(self):
+        pv = qk = 0
+        o_seg = -1
+        while pv < self.T:
+            issued = False
+            if pv < qk and self.p_full[pv % STAGES].passes(self.p_full_phase(pv)):
+                s = pv % STAGES
+                self.pipe.append(("PV", pv, self.seg_of[pv] != o_seg))
+                o_seg = self.seg_of[pv]
+                self.pipe.append(("commit", self.kv_empty[s], pv // STAGES))
+                if self.mut == "single_pv_barrier":
+                    self.pipe.append(("commit", self.pv_bar, pv))
+                pv += 1
+                issued = True
+            if qk < self.T:
+                s, sb = qk % STAGES, qk & 1
+                first = qk in self.first_of_seg
+                if (self.kv_full[s].passes(qk // STAGES)
+                        and (not first or self.q_full.passes(self.seg_of[qk]))
+                        and self.s_empty[sb].passes((qk >> 1) - 1)):
+                    self.pipe.append(("QK", qk))
+                    self.pipe.append(("commit", self.s_full[sb], qk >> 1))
+                    qk += 1
+                    issued = True
+            yield ("step",) if issued else ("idle",)
+
+    def softmax(self, w):
+        live = w < self.plan.live_warps
+        self._stage_q(w, 0)
+        yield ("step",)
+        self.q_full.arrive(0)
+        t = 0
+        for k, n in enumerate(self.plan.segments):
+            any_pv = False
+            for j in range(n):
+                s, sb = t % STAGES, t & 1
+                yield ("wait", lambda s=s, t=t: self.kv_full[s].passes(t // STAGES))
+                yield ("wait", lambda sb=sb, t=t: self.s_full[sb].passes(t >> 1))
+                if live:
+                    if self.st.s_page[sb] != t:
+                        raise ProtocolError(f"softmax {w} reads S[{sb}] for page {t}, holding {self.st.s_page[sb]}")
+                    self.st.s_reading[sb].add(w)
+                    yield ("step",)
+                    self.st.s_reading[sb].discard(w)
+                self.s_empty[sb].arrive(t >> 1)
+                need = live and any_pv and bool((self.plan.rescale or {}).get((w, t), False))
+                if need:
+                    if self.mut != "no_rescale_wait":
+                        yield ("wait", lambda t=t: self.kv_empty[(t - 1) % STAGES].passes((t - 1) // STAGES))
+                    if (t - 1) not in self.st.pv_done:
+                        raise ProtocolError(f"softmax {w} rescales O before PV of page {t - 1} completed")
+                    self.st.o_busy.add(w)
+                    yield ("step",)
+                    self.st.o_busy.discard(w)
+                if live:
+                    if t not in self.st.qk_done or self.st.stage_page[s] != t:
+                        raise ProtocolError(f"softmax {w} writes P of page {t} into a stage QK still reads")
+                    yield ("step",)
+                    self.st.p_written[t] = self.st.p_written.get(t, 0) + 1
+                self.p_full[s].arrive(self.p_full_phase(t))
+                any_pv = True
+                if j == n - 1:
+                    if k + 1 < len(self.plan.segments):
+                        if t not in self.st.qk_done:
+                            raise ProtocolError(f"softmax {w} overwrites the query tile while QK of page {t} runs")
+                        self._stage_q(w, k + 1)
+                        yield ("step",)
+                        self.q_full.arrive(k + 1)
+                    if live:
+                        if self.mut == "single_pv_barrier":
+                            yield ("wait", lambda t=t: self.pv_bar.passes(t))
+                        else:
+                            yield ("wait", lambda s=s, t=t: self.kv_empty[s].passes(t // STAGES))
+                        if t not in self.st.pv_done:
+                            raise ProtocolError(f"softmax {w} reads O for segment {k} before PV of page {t} completed")
+                        self.st.o_busy.add(w)
+                        yield ("step",)
+                        self.st.o_busy.discard(w)
+                    self.st.epilogue_done[k] = self.st.epilogue_done.get(k, 0) + 1
+                t += 1
+
+    # -- helpers ---------------------------------------------------------------
+    def _stage_write_begin(self, s, t):
+        prev = self.st.stage_page[s]
+        if prev is not None and prev != t and prev not in self.st.pv_done:
+            raise ProtocolError(f"page {t} overwrites stage {s} while page {prev} is still in use")
+
+    def _stage_write_end(self, s, t):
+        self.st.stage_writers[s] += 1
+        if self.st.stage_writers[s] == GATHER_WARPS:
+            self.st.stage_writers[s] = 0
+            self.st.stage_page[s] = t
+
+    def _stage_q(self, w, seg):
+        self.st.q_writes[seg] = self.st.q_writes.get(seg, 0) + 1
+        if self.st.q_writes[seg] == WARPS:
+            self.st.q_seg = seg
+
+    def _land(self, t):
+        s = t % STAGES
+        self.st.stage_page[s] = t
+        self.kv_full[s].arrive(t // STAGES)
+
+    def _pipe_pop(self):
+        item = self.pipe.pop(0)
+        kind = item[0]
+        if kind == "commit":
+            item[1].arrive(item[2])
+        elif kind == "QK":
+            t = item[1]
+            s, sb = t % STAGES, t & 1
+            if self.st.stage_page[s] != t:
+                raise ProtocolError(f"QK of page {t} reads stage {s} holding {self.st.stage_page[s]}")
+            if self.st.q_seg != self.seg_of[t]:
+                raise ProtocolError(f"QK of page {t} reads the query tile of segment {self.st.q_seg}")
+            if self.st.s_reading[sb]:
+                raise ProtocolError(f"QK of page {t} overwrites S[{sb}] while it is being read")
+            self.st.s_page[sb] = t
+            self.st.qk_done.add(t)
+        else:
+            t, first = item[1], item[2]
+            s = t % STAGES
+            if self.st.stage_page[s] != t:
+                raise ProtocolError(f"PV of page {t} reads stage {s} holding {self.st.stage_page[s]}")
+            if self.st.p_written.get(t, 0) != self.plan.live_warps:
+                raise ProtocolError(f"PV of page {t} reads P before every live warp wrote it")
+            if self.st.o_busy:
+                raise ProtocolError(f"PV of page {t} updates O while warps {sorted(self.st.o_busy)} use it")
+            seg = self.seg_of[t]
+            if first and seg > 0 and self.st.epilogue_done.get(seg - 1, 0) != WARPS:
+                raise ProtocolError(f"PV of page {t} restarts O before the epilogue of segment {seg - 1}")
+            self.st.pv_done.add(t)
+
+    # -- scheduler -------------------------------------------------------------
+    def run(self, max_steps: int = 200000):
+        roles = [self.mma()] + [self.softmax(w) for w in range(WARPS)]
+        roles += [self.gather(g) for g in range(GATHER_WARPS)] if self.plan.fp8 else [self.producer()]
+        waiting = [None] * len(roles)        # pending wait predicate, or "idle"
+        done = [False] * len(roles)
+
+        def advance(i):
+            try:
+                cmd = next(roles[i])
+            except StopIteration:
+                done[i] = True
+                return
+            waiting[i] = cmd[1] if cmd[0] == "wait" else ("idle" if cmd[0] == "idle" else None)
+
+        for i in range(len(roles)):
+            advance(i)
+        for _ in range(max_steps):
+            if all(done) and not self.pipe and not self.loads:
+                return
+            movers, polls = [], []
+            for i in range(len(roles)):
+                if done[i]:
+                    continue
+                w = waiting[i]
+                if w == "idle":
+                    polls.append(("role", i))
+                elif w is None or w():
+                    movers.append(("role", i))
+            if self.pipe:
+                movers.append(("pipe", None))
+            movers += [("land", t) for t in self.loads]
+            if not movers:
+                if not polls:
+                    raise ProtocolError("deadlock: no role can move and nothing is in flight")
+                i = polls[0][1]
+                pipe_before = len(self.pipe)
+                advance(i)
+                if waiting[i] == "idle" and len(self.pipe) == pipe_before:
+                    raise ProtocolError("deadlock: the MMA warp polls, nothing else can move")
+                continue
+            kind, arg = self.rng.choice(movers + polls)
+            if kind == "role":
+                advance(arg)
+            elif kind == "pipe":
+                self._pipe_pop()
+            else:
+                self.loads.remove(arg)
+                self._land(arg)
+        raise ProtocolError("no completion within the step budget")
