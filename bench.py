@@ -136,6 +136,24 @@ def whole_job_rates(kv_bytes: int, flops: int, world: int, ms_step: float):
     return kv_bytes * world / (ms_step * 1e-3) / 1e9, flops * world / (ms_step * 1e-3) / 1e12
 
 
+def attention_roofline(kv_bytes: int, flops: int, attn_ms: float, hbm_gbs: float, tc_burst: float,
+                       tc_sustained: float) -> dict:
+    """Roofline of the attention kernel: the resource whose roofline time is
+    longer bounds it -- KV bytes at the measured copy bandwidth, or FLOPs at
+    the measured bf16 GEMM rate.  The timed loop runs back to back for
+    seconds, like the sustained GEMM measurement, so that figure is the
+    tensor peak (the burst fraction is reported beside it)."""
+    gbs = kv_bytes / (attn_ms * 1e-3) / 1e9
+    tfs = flops / (attn_ms * 1e-3) / 1e12
+    if flops / (tc_sustained * 1e12) > kv_bytes / (hbm_gbs * 1e9):
+        return {"bound": "tensor", "achieved": round(tfs, 1), "peak": tc_sustained, "unit": "TFLOP/s",
+                "frac": round(tfs / tc_sustained, 4), "peak_kind": "sustained bf16 GEMM",
+                "frac_of_burst_peak": round(tfs / tc_burst, 4), "hbm_frac": round(gbs / hbm_gbs, 4)}
+    return {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_gbs, "unit": "GB/s",
+            "frac": round(gbs / hbm_gbs, 4), "peak_kind": "copy bandwidth",
+            "tensor_frac": round(tfs / tc_burst, 4)}
+
+
 def _blas_threads() -> int:
     try:
         import threadpoolctl
@@ -497,21 +515,7 @@ def main():
             torch.distributed.destroy_process_group()
         return 0
 
-    # Roofline of the attention kernel: the resource whose roofline time is
-    # longer bounds it -- KV bytes at the measured copy bandwidth, or FLOPs at
-    # the measured bf16 GEMM rate.  The timed loop runs back to back for
-    # seconds, like the sustained GEMM measurement, so that figure is the
-    # tensor peak (the burst fraction is reported beside it).
-    gbs = kv_bytes / (attn_ms * 1e-3) / 1e9
-    tfs = flops / (attn_ms * 1e-3) / 1e12
-    if flops / (tc_sus * 1e12) > kv_bytes / (hbm * 1e9):
-        roof = {"bound": "tensor", "achieved": round(tfs, 1), "peak": tc_sus, "unit": "TFLOP/s",
-                "frac": round(tfs / tc_sus, 4), "peak_kind": "sustained bf16 GEMM",
-                "frac_of_burst_peak": round(tfs / tc, 4), "hbm_frac": round(gbs / hbm, 4)}
-    else:
-        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(gbs / hbm, 4), "peak_kind": "copy bandwidth",
-                "tensor_frac": round(tfs / tc, 4)}
+    roof = attention_roofline(kv_bytes, flops, attn_ms, hbm, tc, tc_sus)
     roof.update({"traffic": ATTN_TRAFFIC_BYTES.get(args.config), "peak_source": peak_src,
                  "kernel": "mla_decode_kernel", "kernel_ms": round(attn_ms, 5)})
     line = {

@@ -1,0 +1,30 @@
+"""bench.py's roofline bookkeeping (CPU): the bound is the resource whose
+roofline time is longer, and the fractions are the achieved rates over the
+measured peaks.  The expected values are those of bench lines measured on a
+B200 (memory-bound and variable-length workloads)."""
+import pytest
+
+import bench
+
+HBM, TC_BURST, TC_SUS = 6541.5, 1617.9, 1374.1
+
+
+def test_memory_bound_workload_is_hbm_bound():
+    r = bench.attention_roofline(603_979_776, 18_253_611_008, 0.12698, HBM, TC_BURST, TC_SUS)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] == HBM
+    assert r["achieved"] == pytest.approx(4756.5, abs=0.1)
+    assert r["frac"] == pytest.approx(0.7271, abs=1e-4)
+
+
+def test_varlen_workload_is_tensor_bound():
+    r = bench.attention_roofline(313_598_592, 75_821_170_688, 0.13011, HBM, TC_BURST, TC_SUS)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["peak"] == TC_SUS
+    assert r["frac"] == pytest.approx(0.4241, abs=1e-4)
+    assert r["frac_of_burst_peak"] == pytest.approx(r["achieved"] / TC_BURST, abs=1e-3)
+
+
+def test_bound_flips_where_the_roofline_times_cross():
+    # 1 GB at 6541.5 GB/s takes as long as F FLOPs at 1374.1 TFLOP/s
+    f_cross = 1e9 / (HBM * 1e9) * TC_SUS * 1e12
+    assert bench.attention_roofline(10 ** 9, int(f_cross * 0.99), 1.0, HBM, TC_BURST, TC_SUS)["bound"] == "hbm"
+    assert bench.attention_roofline(10 ** 9, int(f_cross * 1.01), 1.0, HBM, TC_BURST, TC_SUS)["bound"] == "tensor"
