@@ -72,7 +72,11 @@ enum {
 #define MLA_DEVERR_INTERNAL 16    /* shared-memory alignment or TMEM allocation problem */
 
 /*
- * Host-only.  Shape of the split plan for one decode step.
+ * Host-only.  Shape of the split plan for one decode step: how many rows the
+ * tile_scheduler_metadata tensor of the metadata call has, and how long
+ * num_splits is ("Was ist FlashMLA?" (topnet.top), section
+ * "2. MLA-Metadaten abrufen": get_mla_metadata returns both; their sizes are
+ * this library's own, the pages do not give them).
  *   batch, s_q, h_q, h_kv : problem sizes (h_kv must be 1)
  *   topk                  : 0 for the dense path, else indices per query token
  *   num_sm_parts          : <= 0 = choose from the current device's SM count;
@@ -104,7 +108,12 @@ MLA_API int mla_get_metadata(const int32_t* cache_seqlens, int batch, int s_q, i
 
 /*
  * Host-only.  Bytes of workspace a decode with this plan needs: fp32 partial
- * outputs and log-sum-exps for at most (units + num_parts) splits.
+ * outputs and log-sum-exps for at most (units + num_parts) splits.  The pages
+ * split the key range through num_splits ("Was ist FlashMLA?" (topnet.top),
+ * sections "2. MLA-Metadaten abrufen" and "3. MLA-Decodierung ausführen")
+ * without saying where partial results live; this scratch is the library's
+ * own.  Returns MLA_ERR_UNSUPPORTED for more than 4 * 65535 query rows per
+ * unit (s_q * h_q dense, h_q sparse), which the combine grid cannot span.
  */
 MLA_API int mla_workspace_bytes(int batch, int s_q, int h_q, int topk, int num_parts, size_t* bytes);
 
@@ -170,9 +179,12 @@ MLA_API int mla_decode_combine(const mla_decode_args* args, void* stream);
  * until the process exits.  A plan needing more than that (see
  * mla_workspace_bytes) returns MLA_ERR_WORKSPACE before anything is
  * launched.  No allocation is made by this call.
- *  - The first call on a device looks the array's device address up with
- *    cudaGetSymbolAddress (once per device, with that device current); make
- *    that first call before any stream capture begins.
+ *  - The first call in a CUDA context looks the array's device address up
+ *    with cudaGetSymbolAddress, with that context current, and keeps it with
+ *    the context's unique id.  A cudaDeviceReset, or a context the caller
+ *    makes current through the driver API, has a new id, so the next call
+ *    looks the address up again (the module and its array may have moved).
+ *    Make the first call in each context before any stream capture begins.
  *  - All calls share the one array, and it keeps whatever the last call left
  *    in it.  Nothing in it needs to start at zero: every slot the combine
  *    kernel reads is written earlier in the same call.  Calls whose kernels
@@ -182,7 +194,6 @@ MLA_API int mla_decode_combine(const mla_decode_args* args, void* stream);
 #define MLA_NOALLOC_SCRATCH_BYTES (64u << 20)
 MLA_API int mla_decode_noalloc(const mla_decode_args* args, void* stream);
 
-/* Human-readable name of a status code (static string). */
 /*
  * FP8 cache writer: quantise n new key rows into the FP8 cache row format
  * (FlashMLA walkthrough (sao.pub), section "二、核心功能与架构": 512 e4m3
@@ -211,6 +222,7 @@ MLA_API int mla_fp8_cache_write(const void* k_new, int64_t k_row_stride, int32_t
                                 void* kv_cache, int64_t k_block_stride, int32_t num_blocks, int32_t* err_word,
                                 void* stream);
 
+/* Human-readable name of a status code (static string). */
 MLA_API const char* mla_status_string(int status);
 
 #ifdef __cplusplus

@@ -86,7 +86,7 @@ namespace {
 
 using namespace dec;
 
-constexpr int kRows = 64;                     // query rows per CTA = M of every MMA
+constexpr int kRows = kTileRows;              // query rows per CTA = M of every MMA
 constexpr int kStages = 3;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemQCol = 128;           // Q tile columns 128..415 in lanes 16-31
@@ -893,9 +893,8 @@ extern "C" __attribute__((visibility("default"))) int mla_trace_clear() {
 }
 #endif
 
-cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, int tile_rows, bool fp8, int row_tiles,
+cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, bool fp8, int row_tiles,
                           cudaStream_t stream) {
-  if (tile_rows != kRows) return cudaErrorInvalidValue;
   return fp8 ? launch_one<true>(p, tmap_kv, row_tiles, stream) : launch_one<false>(p, tmap_kv, row_tiles, stream);
 }
 

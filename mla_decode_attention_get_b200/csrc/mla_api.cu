@@ -6,7 +6,6 @@
 #include <atomic>
 #include <cstdint>
 #include <cmath>
-#include <cstdlib>
 #include <cstring>
 
 #include "mla_decode.h"
@@ -21,31 +20,21 @@ using mla::kPage;
 struct Plan {
   int units;          // sequences (dense) or (sequence, token) pairs (sparse)
   int rows_per_unit;  // s_q * h_q (dense) or h_q (sparse)
-  int tile_rows;      // query rows per CTA (per CTA pair on the two-CTA kernel)
-  int row_tiles;      // row tiles per partition
-  bool pair;          // two-CTA kernel
+  int row_tiles;      // 64-row tiles per unit (one CTA each per partition)
 };
-
-// MLA_TWO_CTA_DECODE=1 in the environment selects the two-CTA kernel for
-// dense units of more than 64 rows (read on every call; the metadata,
-// workspace and decode calls of one step must see the same value).
-bool two_cta_opt_in() {
-  const char* v = std::getenv("MLA_TWO_CTA_DECODE");
-  return v != nullptr && v[0] == '1' && v[1] == '\0';
-}
 
 int make_plan(int batch, int s_q, int h_q, int h_kv, int topk, Plan* pl) {
   if (batch < 1 || s_q < 1 || h_q < 1 || topk < 0) return MLA_ERR_INVALID_ARG;
   if (h_kv != 1) return MLA_ERR_UNSUPPORTED;
   const long long rows = static_cast<long long>(s_q) * h_q;
   const long long units = topk > 0 ? static_cast<long long>(batch) * s_q : batch;
-  if (rows > (1 << 20) || units > (1 << 24)) return MLA_ERR_INVALID_ARG;
+  if (units > (1 << 24)) return MLA_ERR_INVALID_ARG;
+  const long long rows_per_unit = topk > 0 ? h_q : rows;
+  // the combine kernel's grid spans a unit's rows in its y dimension
+  if (rows_per_unit > mla::kMaxRowsPerUnit) return MLA_ERR_UNSUPPORTED;
   pl->units = static_cast<int>(units);
-  pl->rows_per_unit = topk > 0 ? h_q : static_cast<int>(rows);
-  const bool opt_in = two_cta_opt_in();
-  pl->pair = mla::use_pair_kernel(pl->rows_per_unit, topk > 0, opt_in);
-  pl->tile_rows = mla::tile_rows_for(pl->rows_per_unit, topk > 0, opt_in);
-  pl->row_tiles = (pl->rows_per_unit + pl->tile_rows - 1) / pl->tile_rows;
+  pl->rows_per_unit = static_cast<int>(rows_per_unit);
+  pl->row_tiles = (pl->rows_per_unit + mla::kTileRows - 1) / mla::kTileRows;
   return MLA_OK;
 }
 
@@ -72,9 +61,7 @@ size_t lse_region_bytes(const Plan& pl, int num_parts) {
 size_t workspace_need(const Plan& pl, int num_parts) {
   const size_t splits = static_cast<size_t>(pl.units) + static_cast<size_t>(num_parts);
   const size_t o_bytes = splits * pl.rows_per_unit * kDv * sizeof(float);
-  const size_t ring = pl.pair ? static_cast<size_t>(num_parts) * pl.row_tiles * mla::kPairSlots * mla::kPairSlotBytes
-                              : 0;
-  return o_bytes + lse_region_bytes(pl, num_parts) + ring;
+  return o_bytes + lse_region_bytes(pl, num_parts);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -153,7 +140,6 @@ int prepare(const mla_decode_args* a, Plan* pl, mla::DecodeParams* kp) {
   const size_t splits = static_cast<size_t>(pl->units) + static_cast<size_t>(a->num_parts);
   kp->ws_o = static_cast<float*>(a->workspace);
   kp->ws_lse = kp->ws_o + splits * pl->rows_per_unit * kDv;
-  kp->ws_pring = pl->pair ? reinterpret_cast<uint8_t*>(kp->ws_lse) + lse_region_bytes(*pl, a->num_parts) : nullptr;
   kp->err = a->err_word;
   kp->batch = a->batch;
   kp->s_q = a->s_q;
@@ -179,10 +165,8 @@ int mla_metadata_shape(int batch, int s_q, int h_q, int h_kv, int topk, int num_
     int sms = 0;
     st = device_sm_count(&sms);
     if (st != MLA_OK) return st;
-    // one partition per SM (per row tile), or per co-resident CTA pair
-    const int slots = pl.pair ? mla::pair_cluster_capacity() : sms;
-    if (slots < 1) return MLA_ERR_CUDA;
-    parts = slots / pl.row_tiles;
+    // one CTA per SM: a partition per SM and row tile
+    parts = sms / pl.row_tiles;
     if (parts < 1) parts = 1;
   }
   if (parts > (1 << 16)) return MLA_ERR_INVALID_ARG;
@@ -222,8 +206,7 @@ int mla_decode_attention(const mla_decode_args* a, void* stream) {
                                      uint64_t(kDqk) * 2, uint64_t(a->k_block_stride), kPage))
     return MLA_ERR_CUDA;
   const cudaError_t e =
-      pl.pair ? mla::launch_decode_pair(kp, tkv, pl.row_tiles, static_cast<cudaStream_t>(stream))
-              : mla::launch_decode(kp, tkv, pl.tile_rows, a->is_fp8 != 0, pl.row_tiles, static_cast<cudaStream_t>(stream));
+      mla::launch_decode(kp, tkv, a->is_fp8 != 0, pl.row_tiles, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

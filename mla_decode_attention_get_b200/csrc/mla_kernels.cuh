@@ -17,25 +17,14 @@ constexpr int kFp8Row = 656;
 constexpr int kMdWords = 8;
 constexpr int kFixedSplitCost = 5;
 
-// Row tile of the decode: the number of (token, head) query rows one CTA (or
-// one CTA pair) handles, the M of every tensor-core MMA; units with fewer
-// rows leave the rest of the tile as zero padding.  The default is the
-// single-CTA kernel with 64-row tiles.  The two-CTA kernel (128-row tiles)
-// serves dense units of more than 64 rows when the caller opts in (it is
-// slower on this hardware today).
-__host__ __device__ constexpr bool use_pair_kernel(int rows_per_unit, bool sparse, bool two_cta_opt_in) {
-  return two_cta_opt_in && !sparse && rows_per_unit > 64;
-}
-__host__ __device__ constexpr int tile_rows_for(int rows_per_unit, bool sparse, bool two_cta_opt_in) {
-  return use_pair_kernel(rows_per_unit, sparse, two_cta_opt_in) ? 128 : 64;
-}
+// Row tile of the decode: the number of (token, head) query rows one CTA
+// handles, the M of every tensor-core MMA; units with fewer rows leave the
+// rest of the tile as zero padding.
+constexpr int kTileRows = 64;
 
-// Two-CTA kernel: per cluster, a ring of kPairSlots entries in global memory
-// carries P [128 x 64] bf16, alpha[128] and 1/l[128] from the score CTA to
-// the value CTA, released and handed back in groups of kPairGroup pages.
-constexpr int kPairGroup = 8;
-constexpr int kPairSlots = 2 * kPairGroup;
-constexpr int kPairSlotBytes = 128 * 128 + 2 * 128 * 4;   // 17408
+// Largest query-row count of one unit: the combine kernel's grid covers a
+// unit's rows 4 to a CTA in its y dimension (at most 65535).
+constexpr int kMaxRowsPerUnit = 4 * 65535;
 
 struct DecodeParams {
   const uint16_t* q;          // bf16 bits [batch, s_q, h_q, 576]
@@ -57,7 +46,6 @@ struct DecodeParams {
   float* lse;
   float* ws_o;                // [splits, rows_per_unit, 512]
   float* ws_lse;              // [splits, rows_per_unit]
-  uint8_t* ws_pring;          // two-CTA kernel: [clusters, kPairSlots, kPairSlotBytes]
   int* err;
   int batch, s_q, h_q;
   int rows_per_unit;
@@ -88,13 +76,8 @@ inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 bl
 cudaError_t launch_metadata(const int* seqlens, int batch, int s_q, int topk, int num_units, int num_parts,
                             int* tile_md, int* num_splits, int* err, cudaStream_t stream);
 
-cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, int tile_rows, bool fp8, int row_tiles,
+cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, bool fp8, int row_tiles,
                           cudaStream_t stream);
-
-cudaError_t launch_decode_pair(const DecodeParams& p, const CUtensorMap& tmap_kv, int row_tiles, cudaStream_t stream);
-
-// Clusters of the two-CTA kernel that fit on the current device at once.
-int pair_cluster_capacity();
 
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream);
 

@@ -1,7 +1,9 @@
 // Allocation-free decode entry point: the split-KV partial results live in a
 // file-scope device array of fixed size instead of a caller-provided
 // workspace.  Everything else is the ordinary mla_decode path.
-#include <atomic>
+#include <cudaTypedefs.h>
+
+#include <mutex>
 
 #include "mla_decode.h"
 #include "mla_kernels.cuh"
@@ -11,16 +13,56 @@ namespace {
 // Every GPU that loads the library holds this array until the process exits.
 static __device__ __align__(256) unsigned char g_mla_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
 
-// Device address of the array, looked up once per device.  In host code the
-// array's name is only a stand-in for the symbol, never a device pointer.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename F>
+F driver_entry(const char* name) {
+  void* ptr = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &ptr, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<F>(ptr);
+}
+
+// Unique id of the context current on this thread (0 if none or unknown).
+// A context created after a cudaDeviceReset, or one the caller made current
+// through the driver API, has a new id even where its handle is reused.
+unsigned long long current_context_id() {
+  static const CtxGetCurrentFn get_current = driver_entry<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_entry<CtxGetIdFn>("cuCtxGetId");
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of the array in the current context.  In host code the
+// array's name is only a stand-in for the symbol, never a device pointer:
+// the address is looked up with cudaGetSymbolAddress, once per context, and
+// kept with the context's id (a reset or another context looks it up again).
 void* scratch_address() {
-  static std::atomic<void*> cache[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  void* ptr = cache[dev].load(std::memory_order_acquire);
-  if (ptr != nullptr) return ptr;
+  constexpr int kSlots = 64;
+  static std::mutex mu;
+  static unsigned long long ids[kSlots];
+  static void* ptrs[kSlots];
+  static int next = 0;
+  unsigned long long id = current_context_id();
+  if (id != 0) {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < kSlots; ++i)
+      if (ids[i] == id) return ptrs[i];
+  }
+  void* ptr = nullptr;
   if (cudaGetSymbolAddress(&ptr, g_mla_noalloc_scratch) != cudaSuccess || ptr == nullptr) return nullptr;
-  cache[dev].store(ptr, std::memory_order_release);
+  if (id == 0) id = current_context_id();     // the lookup may have made the primary context current
+  if (id != 0) {
+    std::lock_guard<std::mutex> lock(mu);
+    ids[next] = id;
+    ptrs[next] = ptr;
+    next = (next + 1) % kSlots;
+  }
   return ptr;
 }
 

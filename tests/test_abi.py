@@ -71,18 +71,16 @@ def test_workspace_bytes(lib):
     assert _abi.workspace_bytes(132, 2, 128, 0, 37) == base
 
 
-def test_workspace_bytes_two_cta(lib, monkeypatch):
-    # opting in to the two-CTA kernel adds, per partition and 128-row tile of
-    # a dense unit of more than 64 rows, a ring of 16 entries of
-    # P [128 x 64] bf16 + 2 x 128 floats
-    monkeypatch.setenv("MLA_TWO_CTA_DECODE", "1")
-    n = _abi.workspace_bytes(132, 2, 128, 0, 37)
-    splits = 132 + 37
-    ring = 37 * 2 * 16 * (128 * 128 + 2 * 128 * 4)
-    assert n == splits * 256 * 512 * 4 + ((splits * 256 * 4 + 255) // 256) * 256 + ring
-    # sparse units and units of at most 64 rows keep the single-CTA kernel
-    assert _abi.workspace_bytes(64, 1, 128, 2048, 74) == (64 + 74) * 128 * 2048 + ((138 * 128 * 4 + 255) // 256) * 256
-    assert _abi.workspace_bytes(128, 1, 64, 0, 148) == (128 + 148) * 64 * 2048 + ((276 * 64 * 4 + 255) // 256) * 256
+def test_row_counts_beyond_the_combine_grid_are_unsupported(lib):
+    # the combine kernel covers a unit's rows 4 to a CTA in grid y (<= 65535)
+    assert _abi.metadata_shape(1, 1, 4 * 65535, 1, 0, 8) == (8, 2)
+    with pytest.raises(_abi.MlaError) as e:
+        _abi.metadata_shape(1, 1, 4 * 65535 + 1, 1, 0, 8)
+    assert e.value.status == _abi.MLA_ERR_UNSUPPORTED
+    with pytest.raises(_abi.MlaError) as e:
+        _abi.workspace_bytes(1, 2, 4 * 65535, 0, 8)             # dense rows = s_q * h_q
+    assert e.value.status == _abi.MLA_ERR_UNSUPPORTED
+    assert _abi.workspace_bytes(1, 2, 4 * 65535, 64, 8) > 0     # sparse rows = h_q
 
 
 def test_decode_rejects_bad_arguments_before_launch(lib):
