@@ -14,6 +14,13 @@ With N > 1 (torchrun, one process per GPU) every rank decodes its own batch
 (batch-sharded replicas: sequences are independent, there is no exchange);
 `value` is the KV bytes of all ranks over the slowest rank's time.
 
+On one GPU the same line also carries `per_config`: every decode
+configuration (tiny, memory-bound, variable-length, MTP causal, FP8 sparse)
+and three decode shapes next to them (s_q = 3 and 4 MTP, h_q = 64), each
+timed the same way (kernel and step microseconds, TFLOP/s, KV GB/s, the
+attention kernel's roofline fraction against the measured peaks, clocks,
+and a bounded sample of the CPU oracle).
+
 `--impl reference` times the fp64 CPU oracle on a bounded sample of the same
 workload (the project has no other reference implementation).
 """
@@ -37,9 +44,9 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
 # DRAM traffic (read + write bytes) of one attention-kernel launch per
-# workload, from one ncu capture of the current kernel (profiles/); None when
-# the kernel changed since or for workloads not captured.
-ATTN_TRAFFIC_BYTES = {2: 627_871_488, 3: 386_982_656, 5: 121_032_960}
+# workload, from one ncu capture of the current kernels (profiles/); None
+# when a kernel changed since or the workload was not captured.
+ATTN_TRAFFIC_BYTES = {"C1": None, "C2": None, "C3": None, "C4": None, "C5": None}
 
 
 def _env_int(k, d):
@@ -140,17 +147,17 @@ def attention_roofline(kv_bytes: int, flops: int, attn_ms: float, hbm_gbs: float
                        tc_sustained: float) -> dict:
     """Roofline of the attention kernel: the resource whose roofline time is
     longer bounds it -- KV bytes at the measured copy bandwidth, or FLOPs at
-    the measured bf16 GEMM rate.  The timed loop runs back to back for
-    seconds, like the sustained GEMM measurement, so that figure is the
-    tensor peak (the burst fraction is reported beside it)."""
+    the measured bf16 GEMM rate.  The timed loops last milliseconds, so the
+    tensor peak is the burst GEMM figure; the fraction of the sustained
+    (power-capped, seconds-long) figure is reported beside it."""
     gbs = kv_bytes / (attn_ms * 1e-3) / 1e9
     tfs = flops / (attn_ms * 1e-3) / 1e12
-    if flops / (tc_sustained * 1e12) > kv_bytes / (hbm_gbs * 1e9):
-        return {"bound": "tensor", "achieved": round(tfs, 1), "peak": tc_sustained, "unit": "TFLOP/s",
-                "frac": round(tfs / tc_sustained, 4), "peak_kind": "sustained bf16 GEMM",
-                "frac_of_burst_peak": round(tfs / tc_burst, 4), "hbm_frac": round(gbs / hbm_gbs, 4)}
+    if flops / (tc_burst * 1e12) > kv_bytes / (hbm_gbs * 1e9):
+        return {"bound": "tensor", "achieved": round(tfs, 1), "peak": tc_burst, "unit": "TFLOP/s",
+                "frac": round(tfs / tc_burst, 4), "peak_kind": "burst bf16 GEMM (measured)",
+                "frac_of_sustained_peak": round(tfs / tc_sustained, 4), "hbm_frac": round(gbs / hbm_gbs, 4)}
     return {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_gbs, "unit": "GB/s",
-            "frac": round(gbs / hbm_gbs, 4), "peak_kind": "copy bandwidth",
+            "frac": round(gbs / hbm_gbs, 4), "peak_kind": "copy bandwidth (measured)",
             "tensor_frac": round(tfs / tc_burst, 4)}
 
 
@@ -273,6 +280,154 @@ def bench_sparse_prefill(args) -> int:
     return 0
 
 
+# Workloads of the per-configuration record: the five decode configurations,
+# then three decode shapes on the MTP configuration's cache (132 sequences of
+# 16384 tokens): 3 and 4 causal query tokens x 128 heads, and 64 heads x 1
+# token.
+PER_CONFIG = ("C1", "C2", "C3", "C4", "C5", "MTP s_q=3", "MTP s_q=4", "h_q=64")
+DERIVED = {"MTP s_q=3": (3, 128, True, 3003), "MTP s_q=4": (4, 128, True, 3004), "h_q=64": (1, 64, False, 3064)}
+
+
+def _workload_of(key, cache):
+    from mla_decode_attention_get_b200 import inputs as I
+    if key in DERIVED:
+        s_q, h_q, causal, seed = DERIVED[key]
+        base = cache.get("C4") or I.make_config(4)
+        cache["C4"] = base
+        name = f"{key} causal={causal} b=132 h_q={h_q} L=16384 (the MTP configuration's cache)"
+        return I.with_queries(base, name, s_q, h_q, causal=causal, seed=seed)
+    w = I.make_config(int(key[1:]))
+    if key == "C4":
+        cache["C4"] = w
+    return w
+
+
+def _workload_name(key, w):
+    from mla_decode_attention_get_b200 import inputs as I
+    return I.CONFIG_NAMES[int(key[1:])] if key not in DERIVED else w.name
+
+
+class Timed:
+    """One workload resident on the device and timed through the C ABI: the
+    scheduler, attention and combine kernels per step."""
+
+    def __init__(self, w, dev):
+        import torch
+        import mla_decode_attention_get_b200 as M
+        from mla_decode_attention_get_b200 import inputs as I
+        self.w, self.dev = w, dev
+        self.flops, self.kv_bytes = I.flops_and_bytes(w)
+        self.t = I.to_device(w, dev)
+        self.stream = torch.cuda.current_stream(dev)
+        topk = w.topk if w.fp8 else 0
+        parts, _ = M.mla_metadata_shape(w.batch, w.s_q, w.h_q, 1, topk)
+        self.md = torch.empty((parts, 8), dtype=torch.int32, device=dev)
+        self.ns = torch.empty((w.batch * (w.s_q if w.indices is not None else 1) + 1,), dtype=torch.int32,
+                              device=dev)
+        sl = self.t["sl"]
+        self.meta = lambda: M.mla_get_metadata(sl, w.batch, w.s_q, w.h_q, 1, topk, self.md, self.ns)  # noqa: E731
+        self.meta()
+        self.call = M.prepare_decode(self.t["q"], self.t["kv"], self.t["bt"], sl, 512, self.md, self.ns,
+                                     w.softmax_scale, w.causal, w.fp8, self.t["idx"])
+        # workloads smaller than L2 flush it with a 256 MB write before every
+        # step, outside the timed events
+        self.flush = (torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+                      if self.kv_bytes < 256 * 2 ** 20 else None)
+
+    def step(self, ev=None):
+        self.meta()
+        if ev is not None:
+            ev[0].record(self.stream)
+        self.call.attention()
+        if ev is not None:
+            ev[1].record(self.stream)
+        self.call.combine()
+
+    def run(self, steps, warmup, world, uuid):
+        """(ms per step, attention-kernel ms per launch, clock summary)."""
+        import torch
+        for _ in range(warmup):
+            if self.flush is not None:
+                self.flush.zero_()
+            self.step()
+        torch.cuda.synchronize()
+        err = int(self.call._keep[9].item())
+        if err != 0:
+            raise RuntimeError(f"{self.w.name}: device error word {err}")
+        # K steps between a barrier and a device synchronisation on both
+        # sides, one event pair around the whole loop (per-step pairs when L2
+        # is flushed between steps, so that the flushes stay outside)
+        step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(steps)]
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        sampler = ClockSampler(self.dev.index if self.dev.index is not None else 0, uuid)
+        with sampler:
+            whole0 = torch.cuda.Event(enable_timing=True)
+            whole1 = torch.cuda.Event(enable_timing=True)
+            whole0.record(self.stream)
+            for k in range(steps):
+                if self.flush is not None:
+                    self.flush.zero_()
+                    step_ev[k][0].record(self.stream)
+                self.step()
+                if self.flush is not None:
+                    step_ev[k][1].record(self.stream)
+            whole1.record(self.stream)
+            torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        ms_total = (whole0.elapsed_time(whole1) if self.flush is None
+                    else sum(a.elapsed_time(b) for a, b in step_ev))
+        # the attention kernel's own duration: the same K steps again, with an
+        # event pair around every attention launch
+        attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(steps)]
+        torch.cuda.synchronize()
+        for k in range(steps):
+            if self.flush is not None:
+                self.flush.zero_()
+            self.step(attn_ev[k])
+        torch.cuda.synchronize()
+        attn_ms = sum(a.elapsed_time(b) for a, b in attn_ev) / steps
+        return ms_total / steps, attn_ms, sampler.summary()
+
+    def l2_note(self):
+        return ("flushed before every step (256 MB write)" if self.flush is not None
+                else f"inputs larger than L2 ({self.kv_bytes / 1e6:.0f} MB KV)")
+
+
+def _gpu_uuid(dev):
+    import torch
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        return None
+
+
+def per_config_record(key, w, tm, ms_step, attn_ms, clocks, peaks, cpu_budget):
+    hbm, tc, tc_sus, _ = peaks
+    roof = attention_roofline(tm.kv_bytes, tm.flops, attn_ms, hbm, tc, tc_sus)
+    roof["traffic"] = ATTN_TRAFFIC_BYTES.get(key)
+    rec = {
+        "workload": _workload_name(key, w), "batch": w.batch, "s_q": w.s_q, "h_q": w.h_q,
+        "causal": bool(w.causal), "cache": "fp8" if w.fp8 else "bf16", "topk": w.topk,
+        "flops": tm.flops, "kv_bytes": tm.kv_bytes,
+        "kernel": "mla_decode_fp8_kernel" if w.fp8 else "mla_decode_kernel",
+        "kernel_us": round(attn_ms * 1e3, 2), "step_us": round(ms_step * 1e3, 2),
+        "tflops": round(tm.flops / (attn_ms * 1e-3) / 1e12, 1),
+        "kv_gbs": round(tm.kv_bytes / (attn_ms * 1e-3) / 1e9, 1),
+        "step_tflops": round(tm.flops / (ms_step * 1e-3) / 1e12, 1),
+        "roofline": roof, "clocks": clocks, "l2": tm.l2_note(),
+    }
+    if cpu_budget > 0:
+        gbs, tfl, desc, cores = cpu_oracle_sample(w, cpu_budget)
+        rec["cpu_baseline"] = {"value": round(tfl, 6), "unit": "TFLOP/s", "kv_gbs": round(gbs, 4),
+                               "cores": cores, "kind": "oracle", "sample": desc}
+    return rec
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -281,7 +436,14 @@ def main():
     ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--per-config-cpu-budget", type=float, default=4.0,
+                    help="seconds of oracle work per entry of the per-configuration record")
+    ap.add_argument("--batch", type=int, default=0, help="shrink the workload's batch (profiling runs)")
+    ap.add_argument("--seqlen", type=int, default=0, help="shrink the workload's cache length (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true")
+    ap.add_argument("--per-config-steps", type=int, default=0,
+                    help="timed steps per per-configuration entry (default: --steps, at most 300)")
     ap.add_argument("--op", default="decode", choices=["decode", "fp8_cache_write", "sparse_prefill"],
                     help="decode (the step: scheduler + attention + combine), the FP8 cache writer alone, "
                          "or a prefill-shaped sparse call")
@@ -297,7 +459,8 @@ def main():
     local_rank = _env_int("LOCAL_RANK", 0)
 
     from mla_decode_attention_get_b200 import inputs as I
-    hbm, tc, tc_sus, peak_src = load_peaks()
+    peaks = load_peaks()
+    hbm, tc, tc_sus, peak_src = peaks
 
     if args.impl == "reference":
         if rank != 0:
@@ -341,85 +504,24 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    uuid = _gpu_uuid(dev)
 
-    w = I.make_config(args.config)
-    flops, kv_bytes = I.flops_and_bytes(w)
-    t = I.to_device(w, dev)
-
-    stream = torch.cuda.current_stream(dev)
-    parts, _ = M.mla_metadata_shape(w.batch, w.s_q, w.h_q, 1, w.topk if w.fp8 else 0)
-    md = torch.empty((parts, 8), dtype=torch.int32, device=dev)
-    ns = torch.empty((w.batch * (w.s_q if w.fp8 else 1) + 1,), dtype=torch.int32, device=dev)
-    meta = lambda: M.mla_get_metadata(t["sl"], w.batch, w.s_q, w.h_q, 1, w.topk if w.fp8 else 0, md, ns)  # noqa: E731
-    meta()
-    call = M.prepare_decode(t["q"], t["kv"], t["bt"], t["sl"], 512, md, ns, w.softmax_scale, w.causal, w.fp8,
-                            t["idx"])
-    l2_small = kv_bytes < 256 * 2 ** 20
-    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev) if l2_small else None
-
-    def step(ev=None):
-        meta()
-        if ev is not None:
-            ev[0].record(stream)
-        call.attention()
-        if ev is not None:
-            ev[1].record(stream)
-        call.combine()
-
-    for _ in range(args.warmup):
-        if flush is not None:
-            flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    if int(call._keep[9].item()) != 0:
-        raise RuntimeError(f"device error word {int(call._keep[9].item())}")
-
-    # Timed region: K steps between a barrier and a device synchronisation on
-    # both sides, one event pair around the whole loop (per-step pairs when
-    # L2 is flushed between steps, so that the flushes stay outside).
-    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    try:
-        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    except Exception:
-        uuid = None
-    sampler = ClockSampler(dev.index if dev.index is not None else 0, uuid)
-    with sampler:
-        whole0 = torch.cuda.Event(enable_timing=True)
-        whole1 = torch.cuda.Event(enable_timing=True)
-        whole0.record(stream)
-        for k in range(args.steps):
-            if flush is not None:
-                flush.zero_()
-                step_ev[k][0].record(stream)
-            step()
-            if flush is not None:
-                step_ev[k][1].record(stream)
-        whole1.record(stream)
-        torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    if flush is None:
-        ms_total = whole0.elapsed_time(whole1)
+    head_key = f"C{args.config}"
+    wl_cache = {}
+    if args.batch or args.seqlen:
+        # a smaller case of the same recipe: a profiling run, not a bench line
+        w = I.make_config(args.config, batch=args.batch or None, seqlen=args.seqlen or None)
+        args.no_per_config = True
+        head_key = f"C{args.config} (reduced: batch {w.batch}, max length {int(w.cache_seqlens.max())})"
     else:
-        ms_total = sum(a.elapsed_time(b) for a, b in step_ev)
-
-    # The attention kernel's own duration: the same K steps again, with an
-    # event pair around every attention launch.
-    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    torch.cuda.synchronize()
-    for k in range(args.steps):
-        if flush is not None:
-            flush.zero_()
-        step(attn_ev[k])
-    torch.cuda.synchronize()
-    attn_ms = sum(a.elapsed_time(b) for a, b in attn_ev) / args.steps
+        w = _workload_of(head_key, wl_cache)
+    tm = Timed(w, dev)
+    flops, kv_bytes = tm.flops, tm.kv_bytes
+    ms_step, attn_ms, clocks = tm.run(args.steps, args.warmup, world, uuid)
     if world > 1:
-        ms_total = max_over_ranks(ms_total, dev)
-    ms_step = ms_total / args.steps
+        ms_step = max_over_ranks(ms_step, dev)
     value, tflops = whole_job_rates(kv_bytes, flops, world, ms_step)
+    t, stream, flush = tm.t, tm.stream, tm.flush
 
     # ---- end to end through the public API, host buffers, copies in the region
     q_host = t["q"].cpu().pin_memory()
@@ -509,6 +611,9 @@ def main():
         torch.cuda.synchronize()
         e2e_ms = a.elapsed_time(b) / e2e_steps
     e2e_value = kv_bytes * world / (e2e_ms * 1e-3) / 1e9
+    if world > 1:
+        e2e_ms_max = max_over_ranks(e2e_ms, dev)
+        e2e_value = kv_bytes * world / (e2e_ms_max * 1e-3) / 1e9
 
     if rank != 0:
         if world > 1:
@@ -516,29 +621,55 @@ def main():
         return 0
 
     roof = attention_roofline(kv_bytes, flops, attn_ms, hbm, tc, tc_sus)
-    roof.update({"traffic": ATTN_TRAFFIC_BYTES.get(args.config), "peak_source": peak_src,
-                 "kernel": "mla_decode_kernel", "kernel_ms": round(attn_ms, 5)})
+    roof.update({"traffic": ATTN_TRAFFIC_BYTES.get(head_key), "peak_source": peak_src,
+                 "kernel": "mla_decode_fp8_kernel" if w.fp8 else "mla_decode_kernel",
+                 "kernel_ms": round(attn_ms, 5)})
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": I.CONFIG_NAMES[args.config], "config": args.config, "batch": w.batch,
+        "config": {"workload": I.CONFIG_NAMES[args.config] if head_key == f"C{args.config}" else head_key,
+                   "config": args.config, "batch": w.batch,
                    "s_q": w.s_q, "h_q": w.h_q, "seq_len": int(w.cache_seqlens.max()),
-                   "page": 64, "topk": w.topk, "kv_bytes": kv_bytes, "flops": flops,
-                   "l2": ("flushed before every step (256 MB write)" if flush is not None
-                          else f"inputs larger than L2 ({kv_bytes / 1e6:.0f} MB KV)"),
+                   "page": 64, "topk": w.topk, "kv_bytes": kv_bytes, "flops": flops, "l2": tm.l2_note(),
                    "parallelism": f"batch-sharded replicas x{world}"},
         "tflops": round(tflops, 3),
         "roofline": roof,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "mode": e2e_mode},
         "gpu_launches": 3 * args.steps,
-        "clocks": sampler.summary(),
+        "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
         gbs, tfl, desc, cores = cpu_oracle_sample(w, args.cpu_budget)
         line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                                 "sample": desc}
+
+    if world == 1 and not args.no_per_config:
+        # every configuration and shape, one at a time, timed like the headline
+        pc_steps = args.per_config_steps or min(args.steps, 300)
+        cpu_budget = 0.0 if args.no_cpu_baseline else args.per_config_cpu_budget
+        per = {}
+        head_rec = per_config_record(head_key, w, tm, ms_step, attn_ms, clocks, peaks, 0.0)
+        head_rec["cpu_baseline"] = line.get("cpu_baseline")
+        head_rec["steps"] = args.steps
+        head_rec["gpu_launches"] = 3 * args.steps
+        del q_dev, bt_dev, sl_dev, idx_dev, t, tm
+        torch.cuda.empty_cache()
+        for key in PER_CONFIG:
+            if key == head_key:
+                per[key] = head_rec
+                continue
+            wk = _workload_of(key, wl_cache)
+            tk = Timed(wk, dev)
+            ms_k, attn_k, clk = tk.run(pc_steps, args.warmup, 1, uuid)
+            per[key] = per_config_record(key, wk, tk, ms_k, attn_k, clk, peaks, cpu_budget)
+            per[key]["steps"] = pc_steps
+            per[key]["gpu_launches"] = 3 * pc_steps
+            del tk
+            torch.cuda.empty_cache()
+        wl_cache.clear()
+        line["per_config"] = per
     print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

@@ -5,10 +5,8 @@
 // out = sum_t softmax(s)_t * K_t[:512] and lse = ln sum_t exp(s_t)
 // ("Was ist FlashMLA?" (topnet.top), section "3. MLA-Decodierung ausführen":
 // o_i, lse_i = flash_mla_with_kvcache(q, kvcache, block_table,
-// cache_seqlens, dv, metadata, num_splits, causal)).  The sparse variant
-// attends only to the cache positions an indices tensor names, reading FP8
-// rows (512 e4m3 + 4 fp32 scales + 64 bf16 RoPE) -- FlashMLA walkthrough
-// (sao.pub), section "二、核心功能与架构".
+// cache_seqlens, dv, metadata, num_splits, causal)), over the bf16 cache.
+// The FP8 cache (dense and sparse) has its own kernel, decode_fp8_sm100.cu.
 //
 // Design (one CTA = one scheduler partition x one tile of 64 query rows):
 //  * Every MMA has M = 64 query rows.  Per 64-token page:
@@ -33,17 +31,13 @@
 //    = 9 boxes of 64 tokens x 64 dims) into the ring and warms L2 a few pages
 //    (and the next query tile) ahead; warp 1 issues the MMAs; warps 2-5 write
 //    each segment's query tile into TMEM, run the online softmax and the
-//    epilogue.  On the FP8 path warps 6-13 gather the indexed (or, dense,
-//    the paged) rows and dequantise them into the same page layout as f16;
-//    that path's MMAs run on f16 operands.
+//    epilogue.
 //  * The running max only moves when a page's max exceeds it by more than
 //    2^8 (per row); the final division by the row sum uses the same stale
 //    max, so the result is exact.
 //  * Every wait is bounded; on timeout the CTA raises MLA_DEVERR_TIMEOUT,
 //    drains its own copies and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
-#include <cuda_fp8.h>
 
 #include "decode_common.cuh"
 #include "mla_kernels.cuh"
@@ -92,10 +86,8 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemQCol = 128;           // Q tile columns 128..415 in lanes 16-31
 constexpr int kPChunk = kChunks - 1;          // the RoPE chunk of a stage, reused for the page's P tile
 
-constexpr int kWarpLoad = 0, kWarpMma = 1, kWarpSoftmax0 = 2, kWarpDequant0 = 6;
-constexpr int kDequantWarps = 8;              // FP8 path: warp dq converts keys [8 dq, 8 dq + 8)
-constexpr int kThreadsDense = 32 * kWarpDequant0;
-constexpr int kThreadsFp8 = 32 * (kWarpDequant0 + kDequantWarps);
+constexpr int kWarpLoad = 0, kWarpMma = 1, kWarpEnd = 6;   // warps 2-5: softmax
+constexpr int kThreads = 32 * kWarpEnd;
 
 struct Smem {
   // page ring; once QK of a page has completed, the page's RoPE chunk holds
@@ -105,7 +97,7 @@ struct Smem {
   // kv_full[S], kv_empty[S], s_full[2], s_empty[2], q_full, p_full[S], done
   static constexpr int n_bars = 3 * kStages + 6;
   static constexpr int info_off = bar_off + n_bars * 8;
-  static constexpr int info_bytes = kStages * 16;                // per stage: int nvalid; uint16 mask[4]
+  static constexpr int info_bytes = kStages * 16;                // per stage: valid keys of the page
   static constexpr int misc_off = info_off + info_bytes;         // tmem base, abort flag
   static constexpr int total = misc_off + 16;
   static_assert(kv_off % 1024 == 0 && kPageBytes % 1024 == 0 && kChunkBytes % 1024 == 0,
@@ -115,8 +107,7 @@ struct Smem {
 
 struct StageInfo {
   int nvalid;
-  uint16_t mask[4];
-  int pad;
+  int pad[3];
 };
 
 struct Bars {
@@ -141,7 +132,6 @@ __device__ __forceinline__ int64_t q_tile_offset(const DecodeParams& p, const Un
 // ---------------------------------------------------------------------------
 // Warp 0 (one lane): TMA loads of cache pages with L2 warmed kPrefetchPages
 // ahead, and an L2 prefetch of the next segment's query tile.
-template <bool FP8>
 __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition& part, const CUtensorMap* tmap_kv,
                                           uint8_t* smem, Bars bars, StageInfo* info, volatile int* abort_flag) {
   const uint64_t pol_kv = l2_policy_evict_first();
@@ -171,9 +161,7 @@ __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition
       if (segment_bounds(p, part, u + 1, jb2, je2))
         bulk_prefetch_l2(p.q + q_tile_offset(p, unit_info(p, u + 1)), q_bytes);
     }
-    if constexpr (FP8) {
-      return true;
-    } else {
+    {
       const UnitInfo ui = unit_info(p, u);
       // read the first pages' table entries together, then warm L2
       const int jn = min(je, jb + kPrefetchPages);
@@ -227,184 +215,6 @@ __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition
 }
 
 // ---------------------------------------------------------------------------
-// Warps 6-13 (FP8 sparse path): gather the rows the indices name, dequantise
-// NoPE (e4m3 x per-128 scale) and convert RoPE into the f16 swizzled page
-// tile (the FP8 path runs its MMAs on f16 operands: the e4m3 codes convert
-// to f16 exactly and one packed multiply applies the scale).
-// Warp dq owns keys [8 dq, 8 dq + 8) of every tile; lane l (< 8) resolves key
-// 8 dq + l (index -> block table -> row).  The next tile's table entries and
-// the index after it are read, and the next rows warmed in L2, while the
-// current tile converts: lane l converts NoPE dims [8 l, 8 l + 8) and
-// [256 + 8 l, 256 + 8 l + 8) and, for l < 16, RoPE dims [512 + 4 l, +4) of
-// each of the warp's 8 rows.
-__device__ __forceinline__ void dequant_role(const DecodeParams& p, const Partition& part, uint8_t* smem,
-                                             Bars bars, StageInfo* info, volatile int* abort_flag, int dq) {
-  const int lane = threadIdx.x & 31;
-  const int kl = lane & 7;
-  bool ok = true;
-
-  // Position of this lane's key in the tile a cursor points at: the index
-  // the indices tensor names (-1 past topk), or, with no indices (the dense
-  // FP8 path), the tile's own cache position (positions >= L are padding).
-  const bool sparse = p.indices != nullptr;
-  auto fetch_pos = [&](const Cursor& c) -> int {
-    if (!c.valid) return -1;
-    const int pos_i = kPage * c.j + 8 * dq + kl;
-    if (!sparse) return pos_i;
-    const bool in = pos_i < p.topk;
-    return ld_nc_s32_if(p.indices + (in ? static_cast<int64_t>(c.u) * p.topk + pos_i : 0), in, -1);
-  };
-  auto row_ptr = [&](int phys, int pos) -> const uint8_t* {
-    return p.kv + static_cast<int64_t>(phys) * p.kv_block_stride + (pos & 63) * kFp8Row;
-  };
-
-  // Loads behind resolving a tile: the length of its unit (as stored: a
-  // negative length admits no position) and the table entry of this lane's
-  // key, issued together (the entry speculatively) and first read a tile later.
-  struct Pending {
-    int pos, L, page_entry;
-  };
-  auto start_resolve = [&](const Cursor& c, int pos) -> Pending {
-    Pending r{pos, 0, -1};
-    if (!c.valid) return r;
-    const int b = sparse ? c.u / p.s_q : c.u;
-    r.L = ld_nc_s32_if(p.seqlens + b, true, 0);
-    const int j = pos >> 6;
-    const bool in = pos >= 0 && j < p.bt_width;
-    r.page_entry = ld_nc_s32_if(p.block_table + (in ? static_cast<int64_t>(b) * p.bt_stride + j : 0), in, -1);
-    return r;
-  };
-  auto finish_resolve = [&](const Cursor& c, const Pending& r, int& phys) -> bool {
-    phys = -1;
-    if (!c.valid) return false;
-    bool v = r.pos >= 0 && r.pos < r.L;
-    if (!v && r.pos != -1 && sparse && lane < 8) atomicOr(p.err, kErrIndex);
-    if (v) {
-      phys = r.page_entry;
-      if (phys < 0 || phys >= p.num_blocks) {
-        if (lane < 8) atomicOr(p.err, kErrBlockTable);
-        v = false;
-      }
-    }
-    return v;
-  };
-
-  // Pipeline over tiles: while tile t converts, the rows of tile t+1 are
-  // warmed in L2, the table entry of tile t+2 and the index of tile t+3 are
-  // in flight.
-  Cursor cur = cursor_begin(p, part);
-  Cursor nxt = cur;
-  cursor_next(p, part, nxt);
-  Cursor nxt2 = nxt;
-  cursor_next(p, part, nxt2);
-  int pos_c = fetch_pos(cur);
-  int phys_c = -1;
-  bool valid_c = finish_resolve(cur, start_resolve(cur, pos_c), phys_c);
-  int pos_n = fetch_pos(nxt);
-  Pending pend_n = start_resolve(nxt, pos_n);
-  int pos_nn = fetch_pos(nxt2);
-  int t = 0;
-  while (cur.valid) {
-    const int s = t % kStages;
-    int phys_n = -1;
-    const bool valid_n = finish_resolve(nxt, pend_n, phys_n);
-    if (valid_n) {
-      // the row of key (lane & 7) spans at most 7 lines; lane group lane >> 3
-      // warms lines g and g + 4 of it
-      const uintptr_t a = reinterpret_cast<uintptr_t>(row_ptr(phys_n, pos_n));
-      const uintptr_t first = a >> 7, last = (a + kFp8Row - 1) >> 7;
-      const uintptr_t g = static_cast<uintptr_t>(lane >> 3);
-      if (first + g <= last) prefetch_line_l2(reinterpret_cast<const void*>((first + g) << 7));
-      if (first + g + 4 <= last) prefetch_line_l2(reinterpret_cast<const void*>((first + g + 4) << 7));
-    }
-    const Pending pend_nn = start_resolve(nxt2, pos_nn);
-    Cursor nxt3 = nxt2;
-    cursor_next(p, part, nxt3);
-    const int pos_nnn = fetch_pos(nxt3);
-    if (!mbar_wait(&bars.kv_empty[s], ((t / kStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
-    if (lane == 0 && dq == 0) MLA_TRACE_EV(0, t);
-    uint8_t* stage = smem + Smem::kv_off + s * kPageBytes;
-    {
-      uint2 n0[8], n1[8], rp[8];
-      float s0[8], s1[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int ki = e;
-        const int phys = __shfl_sync(0xffffffffu, phys_c, ki);
-        const int pos = __shfl_sync(0xffffffffu, pos_c, ki);
-        const bool v = __shfl_sync(0xffffffffu, valid_c ? 1 : 0, ki) != 0;
-        n0[e] = n1[e] = rp[e] = make_uint2(0, 0);
-        s0[e] = s1[e] = 0.f;
-        if (v) {
-          const uint8_t* row = row_ptr(phys, pos);
-          n0[e] = __ldg(reinterpret_cast<const uint2*>(row + 8 * lane));
-          n1[e] = __ldg(reinterpret_cast<const uint2*>(row + 256 + 8 * lane));
-          s0[e] = __ldg(reinterpret_cast<const float*>(row + 512 + 4 * (lane >> 4)));
-          s1[e] = __ldg(reinterpret_cast<const float*>(row + 520 + 4 * (lane >> 4)));
-          if (lane < 16) rp[e] = __ldg(reinterpret_cast<const uint2*>(row + 528 + 8 * lane));
-        }
-      }
-      if (lane == 0 && dq == 0) MLA_TRACE_EV(1, t);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int k = 8 * dq + e;   // token row of the tile
-        const int sw = k & 7;
-        const uint32_t slot = static_cast<uint32_t>(((lane & 7) ^ sw) << 4);
-        const uint32_t rowa = smem_u32(stage + k * 128);
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          // e4m3 pairs convert exactly to f16 pairs; one packed f16 multiply
-          // applies the block scale (rounded once, to 11 significant bits)
-          const uint2 codes = half ? n1[e] : n0[e];
-          const float sc = half ? s1[e] : s0[e];
-          const uint32_t sc2 = pack_f16x2(sc, sc);
-          const uint32_t w[2] = {codes.x, codes.y};
-          uint32_t o[4];
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] & 0xFFFFu), __NV_E4M3);
-            const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] >> 16), __NV_E4M3);
-            o[2 * i] = hmul2_f16(*reinterpret_cast<const uint32_t*>(&lo), sc2);
-            o[2 * i + 1] = hmul2_f16(*reinterpret_cast<const uint32_t*>(&hi), sc2);
-          }
-          const int chunk = 4 * half + (lane >> 3);
-          st_shared_v4(rowa + chunk * kChunkBytes + slot, make_uint4(o[0], o[1], o[2], o[3]));
-        }
-        if (lane < 16) {
-          // RoPE dims arrive as bf16: to f16 like the rest of the tile
-          const uint32_t unit = static_cast<uint32_t>(((lane >> 1) ^ sw) << 4) + (lane & 1) * 8;
-          asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(rowa + 8 * kChunkBytes + unit),
-                       "r"(bf16x2_to_f16x2(rp[e].x)), "r"(bf16x2_to_f16x2(rp[e].y))
-                       : "memory");
-        }
-      }
-    }
-    const uint32_t mask = __ballot_sync(0xffffffffu, valid_c) & 0xFFu;
-    if (lane == 0) reinterpret_cast<uint8_t*>(info[s].mask)[dq] = static_cast<uint8_t>(mask);
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bars.kv_full[s]);
-    if (lane == 0 && dq == 0) MLA_TRACE_EV(15, t);
-    cur = nxt;
-    nxt = nxt2;
-    nxt2 = nxt3;
-    pos_c = pos_n;
-    phys_c = phys_n;
-    valid_c = valid_n;
-    pos_n = pos_nn;
-    pend_n = pend_nn;
-    pos_nn = pos_nnn;
-    ++t;
-  }
-  if (!ok && lane == 0) raise_abort(abort_flag, p.err);
-}
-
-__device__ __forceinline__ int stage_nvalid(const StageInfo& si, bool fp8) {
-  if (!fp8) return si.nvalid;
-  return __popc(si.mask[0]) + __popc(si.mask[1]) + __popc(si.mask[2]) + __popc(si.mask[3]);
-}
-
-// ---------------------------------------------------------------------------
 // Warp 1 (whole warp, one elected lane issues): the QK^T and PV MMAs.  Lane 0
 // tests the barriers and broadcasts, so control flow stays warp-uniform and
 // the MMA operands stay uniform.  Two cursors walk the pages: QK(t)
@@ -412,12 +222,11 @@ __device__ __forceinline__ int stage_nvalid(const StageInfo& si, bool fp8) {
 // softmax has written P(t).  Whichever is ready goes first (PV preferred, as
 // it releases the page's stage), so a late page never holds back the PV of
 // the previous one.
-template <bool FP8>
 __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition& part, uint8_t* smem, Bars bars,
                                          const StageInfo* info, uint32_t tmem_base, volatile int* abort_flag) {
-  // S = Q K^T and O += P V (V MN-major); the FP8 path runs on f16 operands
-  constexpr uint32_t idesc_qk = FP8 ? idesc_f16_f32(kRows, kPage, false, false) : idesc_bf16_f32(kRows, kPage, false, false);
-  constexpr uint32_t idesc_pv = FP8 ? idesc_f16_f32(kRows, 256, false, true) : idesc_bf16_f32(kRows, 256, false, true);
+  // S = Q K^T and O += P V (V MN-major)
+  constexpr uint32_t idesc_qk = idesc_bf16_f32(kRows, kPage, false, false);
+  constexpr uint32_t idesc_pv = idesc_bf16_f32(kRows, 256, false, true);
   const uint32_t tmem_q = tmem_base + (16u << 16) + kTmemQCol;   // A operand of QK (lanes 16-31)
   // descriptors of stage 0; a stage's own add its offset to the 16-B address field
   const uint32_t ring = smem_u32(smem + Smem::kv_off);
@@ -477,7 +286,7 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
           ready(&bars.s_empty[sb], ((qk.t >> 1) & 1) ^ 1)) {
         if (lane == 0) MLA_TRACE_EV(2, qk.t);
         tc_fence_after();
-        const int nv = stage_nvalid(info[s], FP8);
+        const int nv = info[s].nvalid;
         qk_nv[s] = nv;
         if (nv > 0) {
           const uint64_t kd = k_desc0 + ((s * kPageBytes) >> 4);
@@ -520,10 +329,8 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
 
 // ---------------------------------------------------------------------------
 // Warps 2-5 (whole warps): the query tile of a unit into TMEM lanes 16-31 as
-// packed bf16 pairs (f16 pairs on the FP8 path).  Thread (r, half) writes
-// row r's dims [128 c + 64 half, +64) for c = 0..3 and RoPE dims
-// [512 + 32 half, +32).
-template <bool F16>
+// packed bf16 pairs.  Thread (r, half) writes row r's dims
+// [128 c + 64 half, +64) for c = 0..3 and RoPE dims [512 + 32 half, +32).
 __device__ __forceinline__ void write_q_tile(const DecodeParams& p, const UnitInfo& ui, uint32_t tq_lane, int r,
                                              int half) {
   const bool valid = r < tile_valid_rows(p);
@@ -538,10 +345,6 @@ __device__ __forceinline__ void write_q_tile(const DecodeParams& p, const UnitIn
     for (int i = 0; i < 8; ++i) {
       v[4 * i] = buf[i].x; v[4 * i + 1] = buf[i].y; v[4 * i + 2] = buf[i].z; v[4 * i + 3] = buf[i].w;
     }
-    if (F16) {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = bf16x2_to_f16x2(v[i]);
-    }
     tmem_st_16x32bx2_x32u(tq_lane + 64 * c, v);
   }
   uint32_t w[16];
@@ -550,16 +353,11 @@ __device__ __forceinline__ void write_q_tile(const DecodeParams& p, const UnitIn
     const uint4 x = valid ? __ldg(src + 64 + 4 * half + i) : make_uint4(0, 0, 0, 0);
     w[4 * i] = x.x; w[4 * i + 1] = x.y; w[4 * i + 2] = x.z; w[4 * i + 3] = x.w;
   }
-  if (F16) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) w[i] = bf16x2_to_f16x2(w[i]);
-  }
   tmem_st_16x32bx2_x16(tq_lane + 256, w);
 }
 
 // ---------------------------------------------------------------------------
 // Warps 2-5: online softmax per page and the per-segment epilogue.
-template <bool FP8>
 __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partition& part, uint8_t* smem,
                                              Bars bars, const StageInfo* info, uint32_t tmem_base,
                                              volatile int* abort_flag) {
@@ -576,8 +374,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
   const float scale_log2 = p.scale_log2;
   const int h_q = p.h_q, s_q = p.s_q;
   const int tok_dense = grow / h_q;                  // dense path: the row's query token
-  const bool sparse = p.indices != nullptr;        // (the sparse path is always FP8)
-  const bool causal = !sparse && p.causal != 0;
+  const bool causal = p.causal != 0;
   const uint32_t s_taddr = tmem_base + (static_cast<uint32_t>(32 * q4 + 16) << 16);
   const uint32_t o_taddr = tmem_base + (static_cast<uint32_t>(32 * q4) << 16);
   const uint32_t p_row0 = smem_u32(smem + Smem::kv_off + kPChunk * kChunkBytes) + r * 128;
@@ -590,7 +387,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
     for (int u = u_from; u <= part.u1 && u < p.num_units; ++u) {
       int jb, je;
       if (segment_bounds(p, part, u, jb, je)) {
-        write_q_tile<FP8>(p, unit_info(p, u), tq_lane, r, half);
+        write_q_tile(p, unit_info(p, u), tq_lane, r, half);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bars.q_full);
@@ -605,7 +402,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
 
   for_each_segment(p, part, [&](int u, int jb, int je) -> bool {
     const UnitInfo ui = unit_info(p, u);
-    if (!sparse && lane == 0 && q4 == 0 && p.seqlens[ui.b] < 0) atomicOr(p.err, kErrSeqlen);
+    if (lane == 0 && q4 == 0 && p.seqlens[ui.b] < 0) atomicOr(p.err, kErrSeqlen);
     float m_run = -INFINITY, l_run = 0.f;
     bool any_pv = false;
     const int lim = ui.L - s_q + tok_dense + 1;      // causal: keys t < lim are visible
@@ -616,7 +413,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
       if (!mbar_wait(&bars.s_full[sb], (t >> 1) & 1, abort_flag)) { ok = false; return false; }
       if (lane == 0 && q4 == 2) MLA_TRACE_EV(4, t);
       tc_fence_after();
-      const int nv = stage_nvalid(info[s], FP8);
+      const int nv = info[s].nvalid;
       const bool work = nv > 0 && warp_live;
       float x[32];
       if (work) tmem_ld_16x32bx2_x32(s_taddr + sb * kPage, x);
@@ -626,14 +423,8 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
 
       float tmax = -INFINITY;
       if (work) {
-        uint32_t vmask;
-        if (FP8) {
-          vmask = static_cast<uint32_t>(info[s].mask[2 * half]) |
-                  (static_cast<uint32_t>(info[s].mask[2 * half + 1]) << 16);
-        } else {
-          const int nk = min(max(nv - key0, 0), 32);
-          vmask = nk >= 32 ? 0xFFFFFFFFu : ((1u << nk) - 1u);
-        }
+        const int nk = min(max(nv - key0, 0), 32);
+        uint32_t vmask = nk >= 32 ? 0xFFFFFFFFu : ((1u << nk) - 1u);
         if (causal && kPage * j + key0 + 31 >= lim) {
           const int nc = min(max(lim - kPage * j - key0, 0), 32);
           vmask &= nc >= 32 ? 0xFFFFFFFFu : ((1u << nc) - 1u);
@@ -672,7 +463,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
         }
       }
 
-      // P = exp2(s - m) as bf16 (f16 for FP8): this thread's 64-B half of
+      // P = exp2(s - m) as bf16: this thread's 64-B half of
       // row r of the K-major swizzled P tile in the page's RoPE chunk, whose
       // last reader, QK of this page, has completed
       const float m_safe = m_run == -INFINITY ? 0.f : m_run;
@@ -685,7 +476,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
           const float a = fast_exp2(x[2 * i] - m_safe);
           const float b = fast_exp2(x[2 * i + 1] - m_safe);
           lsum += a + b;
-          pk[i] = FP8 ? pack_f16x2(a, b) : pack_bf16x2(a, b);
+          pk[i] = pack_bf16x2(a, b);
         }
         l_run += lsum;
       } else {
@@ -703,7 +494,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
       if (lane == 0 && q4 == 2) MLA_TRACE_EV(13, t);
 
       // a partial last page may hold non-finite padding: zero its unused V rows
-      if (!FP8 && nv > 0 && nv < kPage) {
+      if (nv > 0 && nv < kPage) {
         uint8_t* stage = smem + Smem::kv_off + s * kPageBytes;
         const int nrow = kPage - nv;
         const int tid = (q4 << 5) | lane;
@@ -763,10 +554,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
           if (split) {
             p.ws_lse[static_cast<int64_t>(split_idx) * R + grow] = lse;
           } else {
-            int b, tok, h;
-            if (sparse) { b = ui.b; tok = ui.token; h = grow; }
-            else { b = ui.b; tok = tok_dense; h = grow % h_q; }
-            p.lse[(static_cast<int64_t>(b) * h_q + h) * s_q + tok] = lse;
+            p.lse[(static_cast<int64_t>(ui.b) * h_q + grow % h_q) * s_q + tok_dense] = lse;
           }
         }
         tc_fence_before();
@@ -780,8 +568,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
 }
 
 // ---------------------------------------------------------------------------
-template <bool FP8>
-__global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreadsDense, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     mla_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_kv) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
@@ -804,11 +591,10 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreadsDense, 1)
   if (threadIdx.x == 0) {
     *abort_flag = misaligned ? 1 : 0;
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars.kv_full[s], FP8 ? kDequantWarps : 1);
+      mbar_init(&bars.kv_full[s], 1);
       mbar_init(&bars.kv_empty[s], 1);
       mbar_init(&bars.p_full[s], 4);
       info[s].nvalid = 0;
-      for (int w = 0; w < 4; ++w) info[s].mask[w] = 0;
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.s_full[i], 1);
@@ -818,7 +604,7 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreadsDense, 1)
     mbar_init(bars.done, 1);
     fence_barrier_init();
   }
-  if (warp == kWarpLoad && lane == 0 && !FP8) prefetch_tensormap(&tmap_kv);
+  if (warp == kWarpLoad && lane == 0) prefetch_tensormap(&tmap_kv);
   if (warp == kWarpMma) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -838,13 +624,11 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreadsDense, 1)
 
   if (!*abort_flag) {
     if (warp == kWarpLoad) {
-      if (lane == 0) load_role<FP8>(p, part, &tmap_kv, smem, bars, info, abort_flag);
+      if (lane == 0) load_role(p, part, &tmap_kv, smem, bars, info, abort_flag);
     } else if (warp == kWarpMma) {
-      mma_role<FP8>(p, part, smem, bars, info, tmem_base, abort_flag);
-    } else if (warp >= kWarpSoftmax0 && warp < kWarpDequant0) {
-      softmax_role<FP8>(p, part, smem, bars, info, tmem_base, abort_flag);
-    } else if (FP8) {
-      dequant_role(p, part, smem, bars, info, abort_flag, warp - kWarpDequant0);
+      mma_role(p, part, smem, bars, info, tmem_base, abort_flag);
+    } else {
+      softmax_role(p, part, smem, bars, info, tmem_base, abort_flag);
     }
   }
   tc_fence_before();
@@ -858,7 +642,6 @@ __global__ void __launch_bounds__(FP8 ? kThreadsFp8 : kThreadsDense, 1)
   }
 }
 
-template <bool FP8>
 cudaError_t launch_one(const DecodeParams& p, const CUtensorMap& tkv, int row_tiles, cudaStream_t stream) {
   constexpr int smem = Smem::total;
   // The shared-memory opt-in is per device; remember which devices have it.
@@ -868,12 +651,11 @@ cudaError_t launch_one(const DecodeParams& p, const CUtensorMap& tkv, int row_ti
   if (e != cudaSuccess) return e;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(__atomic_load_n(&configured, __ATOMIC_ACQUIRE) & bit)) {
-    e = cudaFuncSetAttribute(mla_decode_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     __atomic_fetch_or(&configured, bit, __ATOMIC_RELEASE);
   }
-  return launch_dependent(mla_decode_kernel<FP8>, dim3(p.num_parts, row_tiles), dim3(FP8 ? kThreadsFp8 : kThreadsDense), smem, stream,
-                          p, tkv);
+  return launch_dependent(mla_decode_kernel, dim3(p.num_parts, row_tiles), dim3(kThreads), smem, stream, p, tkv);
 }
 
 }  // namespace
@@ -893,9 +675,8 @@ extern "C" __attribute__((visibility("default"))) int mla_trace_clear() {
 }
 #endif
 
-cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, bool fp8, int row_tiles,
-                          cudaStream_t stream) {
-  return fp8 ? launch_one<true>(p, tmap_kv, row_tiles, stream) : launch_one<false>(p, tmap_kv, row_tiles, stream);
+cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, int row_tiles, cudaStream_t stream) {
+  return launch_one(p, tmap_kv, row_tiles, stream);
 }
 
 }  // namespace mla

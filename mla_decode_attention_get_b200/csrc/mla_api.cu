@@ -205,8 +205,9 @@ int mla_decode_attention(const mla_decode_args* a, void* stream) {
   if (!a->is_fp8 && !encode_bf16_map(&tkv, a->k_cache, uint64_t(kPage), uint64_t(a->num_blocks),
                                      uint64_t(kDqk) * 2, uint64_t(a->k_block_stride), kPage))
     return MLA_ERR_CUDA;
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const cudaError_t e =
-      mla::launch_decode(kp, tkv, a->is_fp8 != 0, pl.row_tiles, static_cast<cudaStream_t>(stream));
+      a->is_fp8 ? mla::launch_decode_fp8(kp, pl.row_tiles, cs) : mla::launch_decode(kp, tkv, pl.row_tiles, cs);
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

@@ -76,8 +76,9 @@ inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 bl
 cudaError_t launch_metadata(const int* seqlens, int batch, int s_q, int topk, int num_units, int num_parts,
                             int* tile_md, int* num_splits, int* err, cudaStream_t stream);
 
-cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, bool fp8, int row_tiles,
-                          cudaStream_t stream);
+// The bf16 cache (TMA page loads through tmap_kv) and the FP8 cache.
+cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, int row_tiles, cudaStream_t stream);
+cudaError_t launch_decode_fp8(const DecodeParams& p, int row_tiles, cudaStream_t stream);
 
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream);
 

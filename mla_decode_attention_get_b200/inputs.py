@@ -238,6 +238,15 @@ def make_config(cfg: int, *, batch: Optional[int] = None, seqlen: Optional[int] 
     raise ValueError(f"unknown config {cfg}")
 
 
+def with_queries(w: Workload, name: str, s_q: int, h_q: int, *, causal: bool, seed: int) -> Workload:
+    """The same cache, block table and lengths as ``w`` (dense path) with new
+    seeded N(0,1) bf16 queries of another shape: the multi-token and head-count
+    variants of a configuration without drawing its cache again."""
+    assert w.indices is None
+    q_bits = _normal_bf16(_rngs(seed, 1)[0], (w.batch, s_q, h_q, D_QK))
+    return dataclasses.replace(w, name=name, s_q=s_q, h_q=h_q, causal=causal, seed=seed, q_bits=q_bits)
+
+
 def flops_and_bytes(w: Workload):
     """Algorithmic work of one decode call: 2*(576+512) FLOPs per unmasked
     (query row, key) pair, and 1152 B per visible bf16 cache row or 656 B per

@@ -1,9 +1,8 @@
-"""A host-side model of the decode kernel's synchronisation protocol.
+"""A host-side model of the decode kernels' synchronisation protocols.
 
-Test infrastructure only.  It restates, role by role, the mbarrier hand-offs
-of one CTA of the decode kernel in `csrc/decode_sm100.cu`:
-- the page producer: the TMA warp on the bf16 path, or 8 gather warps on the
-  FP8 path;
+Test infrastructure only.  `Model` restates, role by role, the mbarrier
+hand-offs of one CTA of the bf16 decode kernel in `csrc/decode_sm100.cu`:
+- the page producer, the TMA warp;
 - the MMA warp's event loop;
 - the four softmax warps, with idle padding warps, lazy rescales, segment
   epilogues and query-tile staging.
@@ -28,6 +27,10 @@ catch it:
 - "no_rescale_wait": rescale O without waiting for PV of the previous page;
 - "single_pv_barrier": the epilogue waits for PV through one barrier
   committed per page, with parity t & 1.
+
+`Fp8Model` (at the end) does the same for the FP8 kernel in
+`csrc/decode_fp8_sm100.cu`, whose protocol differs (two stages filled by 8
+gather warps, QK^T in two passes, P' tiles in the stage).
 """
 from __future__ import annotations
 
@@ -37,7 +40,7 @@ from typing import Dict, List, Optional
 
 STAGES = 3
 WARPS = 4            # softmax warps, one per TMEM lane quadrant
-GATHER_WARPS = 8     # FP8 path
+GATHER_WARPS = 8     # FP8 kernel
 
 
 class ProtocolError(AssertionError):
@@ -69,7 +72,7 @@ class Barrier:
 class Plan:
     segments: List[int]                 # pages per segment, in order
     live_warps: int                     # softmax warps with at least one real row
-    fp8: bool = False
+    fp8: bool = False                   # (Fp8Model only)
     rescale: Optional[Dict] = None      # (warp, page) -> bool: a rescale is needed
 
 
@@ -99,7 +102,7 @@ class Model:
             self.seg_of += [k] * n
             t += n
         S = STAGES
-        self.kv_full = [Barrier(f"kv_full[{s}]", GATHER_WARPS if plan.fp8 else 1) for s in range(S)]
+        self.kv_full = [Barrier(f"kv_full[{s}]", 1) for s in range(S)]
         self.kv_empty = [Barrier(f"kv_empty[{s}]", 1) for s in range(S)]
         self.s_full = [Barrier(f"s_full[{b}]", 1) for b in range(2)]
         self.s_empty = [Barrier(f"s_empty[{b}]", WARPS) for b in range(2)]
@@ -125,16 +128,6 @@ class Model:
             yield ("wait", lambda s=s, t=t: self.kv_empty[s].passes(t // STAGES - 1))
             self._stage_write_begin(s, t)
             self.loads.append(t)
-            yield ("step",)
-
-    def gather(self, w):
-        for t in range(self.T):
-            s = t % STAGES
-            yield ("wait", lambda s=s, t=t: self.kv_empty[s].passes(t // STAGES - 1))
-            self._stage_write_begin(s, t)
-            yield ("step",)
-            self._stage_write_end(s, t)
-            self.kv_full[s].arrive(t // STAGES)
             yield ("step",)
 
     def mma(self):
@@ -224,12 +217,6 @@ class Model:
         if prev is not None and prev != t and prev not in self.st.pv_done:
             raise ProtocolError(f"page {t} overwrites stage {s} while page {prev} is still in use")
 
-    def _stage_write_end(self, s, t):
-        self.st.stage_writers[s] += 1
-        if self.st.stage_writers[s] == GATHER_WARPS:
-            self.st.stage_writers[s] = 0
-            self.st.stage_page[s] = t
-
     def _stage_q(self, w, seg):
         self.st.q_writes[seg] = self.st.q_writes.get(seg, 0) + 1
         if self.st.q_writes[seg] == WARPS:
@@ -272,8 +259,7 @@ class Model:
 
     # -- scheduler -------------------------------------------------------------
     def run(self, max_steps: int = 200000):
-        roles = [self.mma()] + [self.softmax(w) for w in range(WARPS)]
-        roles += [self.gather(g) for g in range(GATHER_WARPS)] if self.plan.fp8 else [self.producer()]
+        roles = [self.mma()] + [self.softmax(w) for w in range(WARPS)] + [self.producer()]
         waiting = [None] * len(roles)        # pending wait predicate, or "idle"
         done = [False] * len(roles)
 
@@ -319,4 +305,281 @@ class Model:
             else:
                 self.loads.remove(arg)
                 self._land(arg)
+        raise ProtocolError("no completion within the step budget")
+
+
+# ---------------------------------------------------------------------------
+# The FP8 kernel (`csrc/decode_fp8_sm100.cu`) has its own protocol:
+# - three stages, converted by 8 gather warps (kv_full) and freed by the
+#   commit after PV of their tile (kv_empty);
+# - QK^T in two passes per tile into three TMEM buffers: pass A (groups 0-2,
+#   committed to sa_full) once the tile is in, the query tile is loaded and the
+#   softmax has read pass B of the previous tile (sb_empty); pass B (group 3
+#   and RoPE into buffers 0-1, committed to sb_full and to the stage's qk_done)
+#   once the softmax has read pass A (sa_empty);
+# - the softmax writes the tile's P into the stage's RoPE chunk (which pass B
+#   reads) after pass B has completed, and arrives p_full;
+# - after converting tile t the gather warps rewrite the codes of tile t-1 as
+#   V' (waiting on qk_done: QK^T reads the codes) and arrive v_ready;
+# - the MMA warp issues, in order per tile: pass A(t), pass B(t), PV(t-1), and
+#   PV(t) at the end of a segment; PV waits p_full and v_ready.
+FP8_STAGES = 3
+
+
+class Fp8Model:
+    """Random interleavings of the FP8 kernel's roles; the same checks as
+    `Model`.  `mutation`:
+    - "no_sa_wait": pass B does not wait for the softmax to read pass A;
+    - "early_p": the softmax writes P before pass B has completed;
+    - "early_v": the gather rewrites V' without waiting for qk_done;
+    - "no_seg_end_pv": PV of a segment's last tile waits for the next tile."""
+
+    def __init__(self, plan: Plan, seed: int, mutation: Optional[str] = None):
+        self.plan, self.rng, self.mut = plan, random.Random(seed), mutation
+        self.T = sum(plan.segments)
+        self.seg_of, self.first_of_seg, self.last_of_seg = [], set(), set()
+        t = 0
+        for k, n in enumerate(plan.segments):
+            self.first_of_seg.add(t)
+            self.last_of_seg.add(t + n - 1)
+            self.seg_of += [k] * n
+            t += n
+        S = FP8_STAGES
+        self.kv_full = [Barrier(f"kv_full[{s}]", GATHER_WARPS) for s in range(S)]
+        self.kv_empty = [Barrier(f"kv_empty[{s}]", 1) for s in range(S)]
+        self.p_full = [Barrier(f"p_full[{s}]", WARPS) for s in range(S)]
+        self.qk_done = [Barrier(f"qk_done[{s}]", 1) for s in range(S)]
+        self.v_ready = [Barrier(f"v_ready[{s}]", GATHER_WARPS) for s in range(S)]
+        self.sa_full, self.sa_empty = Barrier("sa_full", 1), Barrier("sa_empty", WARPS)
+        self.sb_full, self.sb_empty = Barrier("sb_full", 1), Barrier("sb_empty", WARPS)
+        self.q_full = Barrier("q_full", WARPS)
+        self.pipe: List[tuple] = []
+        self.stage_page: List[Optional[int]] = [None] * S
+        self.stage_writers = [0] * S
+        self.v_writers = [0] * S
+        self.codes_are_v = [False] * S        # the stage's codes were rewritten as V'
+        self.rope_is_p = [False] * S          # the RoPE chunk holds P (pass B of its tile is over)
+        self.buf = [None, None, None]         # (tile, pass) held by each partial-S buffer
+        self.reading = [set(), set(), set()]
+        self.qka_done, self.qkb_done, self.pv_done = set(), set(), set()
+        self.p_written: Dict[int, int] = {}
+        self.q_writes: Dict[int, int] = {}
+        self.q_seg = -1
+        self.o_busy = set()
+        self.epilogue_done: Dict[int, int] = {}
+
+    # -- roles -------------------------------------------------------------------
+    def gather(self, w):
+        ph = lambda t: t // FP8_STAGES  # noqa: E731
+        tr = 0
+        for t in range(self.T):
+            s = t % FP8_STAGES
+            yield ("wait", lambda s=s, t=t: self.kv_empty[s].passes(ph(t) - 1))
+            prev = self.stage_page[s]
+            if prev is not None and prev != t and prev not in self.pv_done:
+                raise ProtocolError(f"tile {t} overwrites stage {s} while tile {prev} is still in use")
+            yield ("step",)
+            self.stage_writers[s] += 1
+            if self.stage_writers[s] == GATHER_WARPS:
+                self.stage_writers[s] = 0
+                self.stage_page[s] = t
+                self.rope_is_p[s] = False
+                self.codes_are_v[s] = False
+            self.kv_full[s].arrive(ph(t))
+            yield ("step",)
+            while t + 1 - tr > 1:
+                yield from self._rewrite(tr)
+                tr += 1
+        while tr < self.T:
+            yield from self._rewrite(tr)
+            tr += 1
+
+    def _rewrite(self, t):
+        s = t % FP8_STAGES
+        if self.mut != "early_v":
+            yield ("wait", lambda s=s, t=t: self.qk_done[s].passes(t // FP8_STAGES))
+        if self.stage_page[s] != t:
+            raise ProtocolError(f"V' of tile {t} rewrites stage {s} holding {self.stage_page[s]}")
+        if t not in self.qkb_done:
+            raise ProtocolError(f"V' of tile {t} rewrites codes that QK^T still reads")
+        yield ("step",)
+        self.v_writers[s] += 1
+        if self.v_writers[s] == GATHER_WARPS:
+            self.v_writers[s] = 0
+            self.codes_are_v[s] = True
+        self.v_ready[s].arrive(t // FP8_STAGES)
+
+    def mma(self):
+        ph = lambda t: t // FP8_STAGES  # noqa: E731
+        prev = None
+        for t in range(self.T):
+            s = t % FP8_STAGES
+            yield ("wait", lambda s=s, t=t: self.kv_full[s].passes(ph(t)))
+            if t in self.first_of_seg:
+                yield ("wait", lambda t=t: self.q_full.passes(self.seg_of[t]))
+            yield ("wait", lambda t=t: self.sb_empty.passes(t - 1))
+            self.pipe.append(("QKA", t))
+            self.pipe.append(("commit", self.sa_full, t))
+            if self.mut != "no_sa_wait":
+                yield ("wait", lambda t=t: self.sa_empty.passes(t))
+            self.pipe.append(("QKB", t))
+            self.pipe.append(("commit", self.sb_full, t))
+            self.pipe.append(("commit", self.qk_done[s], ph(t)))
+            if prev is not None:
+                yield from self._pv(prev)
+            prev = t
+            if t in self.last_of_seg and self.mut != "no_seg_end_pv":
+                yield from self._pv(t)
+                prev = None
+            yield ("step",)
+        if prev is not None:
+            yield from self._pv(prev)
+
+    def _pv(self, t):
+        s = t % FP8_STAGES
+        yield ("wait", lambda s=s, t=t: self.p_full[s].passes(t // FP8_STAGES))
+        yield ("wait", lambda s=s, t=t: self.v_ready[s].passes(t // FP8_STAGES))
+        self.pipe.append(("PV", t))
+        self.pipe.append(("commit", self.kv_empty[s], t // FP8_STAGES))
+
+    def softmax(self, w):
+        live = w < self.plan.live_warps
+        self._stage_q(0)
+        yield ("step",)
+        self.q_full.arrive(0)
+        t = 0
+        for k, n in enumerate(self.plan.segments):
+            any_pv = False
+            for j in range(n):
+                s = t % FP8_STAGES
+                yield ("wait", lambda s=s, t=t: self.kv_full[s].passes(t // FP8_STAGES))
+                yield ("wait", lambda t=t: self.sa_full.passes(t))
+                if live:
+                    for b in range(3):
+                        if self.buf[b] != (t, "A"):
+                            raise ProtocolError(f"softmax {w} reads buffer {b} for pass A of tile {t}, "
+                                                f"holding {self.buf[b]}")
+                        self.reading[b].add(w)
+                    yield ("step",)
+                    for b in range(3):
+                        self.reading[b].discard(w)
+                self.sa_empty.arrive(t)
+                if self.mut != "early_p":
+                    yield ("wait", lambda t=t: self.sb_full.passes(t))
+                    if live:
+                        for b in range(2):
+                            if self.buf[b] != (t, "B"):
+                                raise ProtocolError(f"softmax {w} reads buffer {b} for pass B of tile {t}, "
+                                                    f"holding {self.buf[b]}")
+                            self.reading[b].add(w)
+                        yield ("step",)
+                        for b in range(2):
+                            self.reading[b].discard(w)
+                    self.sb_empty.arrive(t)
+                need = live and any_pv and bool((self.plan.rescale or {}).get((w, t), False))
+                if need:
+                    yield ("wait", lambda t=t: self.kv_empty[(t - 1) % FP8_STAGES].passes((t - 1) // FP8_STAGES))
+                    if (t - 1) not in self.pv_done:
+                        raise ProtocolError(f"softmax {w} rescales O before PV of tile {t - 1} completed")
+                    self.o_busy.add(w)
+                    yield ("step",)
+                    self.o_busy.discard(w)
+                if live:
+                    if t not in self.qkb_done or self.stage_page[s] != t:
+                        raise ProtocolError(f"softmax {w} writes P of tile {t} into a RoPE chunk pass B still reads")
+                    yield ("step",)
+                    self.rope_is_p[s] = True
+                    self.p_written[t] = self.p_written.get(t, 0) + 1
+                if self.mut == "early_p":
+                    yield ("wait", lambda t=t: self.sb_full.passes(t))
+                    self.sb_empty.arrive(t)
+                self.p_full[s].arrive(t // FP8_STAGES)
+                any_pv = True
+                if j == n - 1:
+                    if k + 1 < len(self.plan.segments):
+                        if t not in self.qkb_done:
+                            raise ProtocolError(f"softmax {w} overwrites the query tile while QK of tile {t} runs")
+                        self._stage_q(k + 1)
+                        yield ("step",)
+                        self.q_full.arrive(k + 1)
+                    if live:
+                        yield ("wait", lambda s=s, t=t: self.kv_empty[s].passes(t // FP8_STAGES))
+                        if t not in self.pv_done:
+                            raise ProtocolError(f"softmax {w} reads O for segment {k} before PV of tile {t} completed")
+                        self.o_busy.add(w)
+                        yield ("step",)
+                        self.o_busy.discard(w)
+                    self.epilogue_done[k] = self.epilogue_done.get(k, 0) + 1
+                t += 1
+
+    def _stage_q(self, seg):
+        self.q_writes[seg] = self.q_writes.get(seg, 0) + 1
+        if self.q_writes[seg] == WARPS:
+            self.q_seg = seg
+
+    def _pipe_pop(self):
+        item = self.pipe.pop(0)
+        kind = item[0]
+        if kind == "commit":
+            item[1].arrive(item[2])
+            return
+        t = item[1]
+        s = t % FP8_STAGES
+        if self.stage_page[s] != t:
+            raise ProtocolError(f"{kind} of tile {t} reads stage {s} holding {self.stage_page[s]}")
+        if kind in ("QKA", "QKB"):
+            if self.q_seg != self.seg_of[t]:
+                raise ProtocolError(f"{kind} of tile {t} reads the query tile of segment {self.q_seg}")
+            if self.codes_are_v[s]:
+                raise ProtocolError(f"{kind} of tile {t} reads codes already rewritten as V'")
+            bufs = (0, 1, 2) if kind == "QKA" else (0, 1)
+            for b in bufs:
+                if self.reading[b]:
+                    raise ProtocolError(f"{kind} of tile {t} overwrites buffer {b} while it is being read")
+            if kind == "QKB" and self.rope_is_p[s]:
+                raise ProtocolError(f"QKB of tile {t} reads a RoPE chunk that holds P")
+            for b in bufs:
+                self.buf[b] = (t, "A" if kind == "QKA" else "B")
+            (self.qka_done if kind == "QKA" else self.qkb_done).add(t)
+        else:
+            if self.p_written.get(t, 0) != self.plan.live_warps:
+                raise ProtocolError(f"PV of tile {t} reads P before every live warp wrote it")
+            if not self.codes_are_v[s]:
+                raise ProtocolError(f"PV of tile {t} reads V' before the gather warps wrote it")
+            if self.o_busy:
+                raise ProtocolError(f"PV of tile {t} updates O while warps {sorted(self.o_busy)} use it")
+            seg = self.seg_of[t]
+            if t in self.first_of_seg and seg > 0 and self.epilogue_done.get(seg - 1, 0) != WARPS:
+                raise ProtocolError(f"PV of tile {t} restarts O before the epilogue of segment {seg - 1}")
+            self.pv_done.add(t)
+
+    def run(self, max_steps: int = 300000):
+        roles = [self.mma()] + [self.softmax(w) for w in range(WARPS)]
+        roles += [self.gather(g) for g in range(GATHER_WARPS)]
+        waiting = [None] * len(roles)
+        done = [False] * len(roles)
+
+        def advance(i):
+            try:
+                cmd = next(roles[i])
+            except StopIteration:
+                done[i] = True
+                return
+            waiting[i] = cmd[1] if cmd[0] == "wait" else None
+
+        for i in range(len(roles)):
+            advance(i)
+        for _ in range(max_steps):
+            if all(done) and not self.pipe:
+                return
+            movers = [("role", i) for i in range(len(roles)) if not done[i] and (waiting[i] is None or waiting[i]())]
+            if self.pipe:
+                movers.append(("pipe", None))
+            if not movers:
+                raise ProtocolError("deadlock: no role can move and nothing is in flight")
+            kind, arg = self.rng.choice(movers)
+            if kind == "role":
+                advance(arg)
+            else:
+                self._pipe_pop()
         raise ProtocolError("no completion within the step budget")

@@ -6,10 +6,10 @@ check that they really rescale.  N(0, 1) data alone never moves a row's max
 past the threshold after the first page, so a few key rows on later pages are
 boosted:
 - bf16 rows are scaled x12;
-- FP8 rows get group scales 2^-5, which is 7-28 times the workload's scales.
-  Every dequantised value (an e4m3 value times a power of two) is then exact
-  in the kernel's f16 operands, so the big logits carry no dequantisation
-  rounding."""
+- FP8 rows either get group scales 2^-5 (7-28 times the workload's scales),
+  or keep their own non-power-of-two scales multiplied by 17 (float32); the
+  second kind is the general case, whose dequantised values have up to 28
+  significant bits, and its boosted logits reach 30-50."""
 from __future__ import annotations
 
 import numpy as np
@@ -29,6 +29,13 @@ def _boost_fp8(w, phys, row):
     w.kv_fp8[phys, row, 0, 512:528] = np.full(4, BOOST_SCALE, "<f4").view(np.uint8)
 
 
+def _boost_fp8_x17(w, phys, row):
+    # the row's own scales x17: not powers of two, so code x scale is not a
+    # short binary number
+    raw = w.kv_fp8[phys, row, 0, 512:528].copy().view("<f4")
+    w.kv_fp8[phys, row, 0, 512:528] = (raw * np.float32(17.0)).astype("<f4").view(np.uint8)
+
+
 def _boost_dense_positions(w, boost):
     for b, L in enumerate(w.cache_seqlens):
         for tok in (700 + b, 1500, int(L) - 3):
@@ -41,16 +48,17 @@ def bf16_case(h_q: int, s_q: int, causal: bool):
     return _boost_dense_positions(w, _boost_bf16)
 
 
-def fp8_dense_case():
+def fp8_dense_case(x17: bool = False):
     w = I.make_workload("fp8dresc", 2, 1, 64, [3000, 2000], fp8=True, seed=47)
-    return _boost_dense_positions(w, _boost_fp8)
+    return _boost_dense_positions(w, _boost_fp8_x17 if x17 else _boost_fp8)
 
 
-def fp8_sparse_case():
+def fp8_sparse_case(x17: bool = False):
     # the rows named at index slots 700 and 1500 of every token
     w = I.make_workload("rescale8", 2, 1, 128, [4000, 3000], fp8=True, topk=2048, seed=53)
+    boost = _boost_fp8_x17 if x17 else _boost_fp8
     for b in range(w.batch):
         for slot in (700, 1500):
             pos = int(w.indices[b, 0, slot])
-            _boost_fp8(w, w.block_table[b, pos // 64], pos % 64)
+            boost(w, w.block_table[b, pos // 64], pos % 64)
     return w

@@ -7,7 +7,7 @@ import pytest
 
 from mla_decode_attention_get_b200 import inputs as I
 from oracle import brute, mla_oracle as O
-from oracle.formats import bf16_bits_to_f64
+from oracle.formats import bf16_bits_to_f64, fp8_rows_to_f64
 
 SCALE = 576 ** -0.5
 
@@ -34,6 +34,40 @@ def test_oracle_matches_brute_force(causal, s_q, lens):
             limit = L - s_q + i + 1 if causal else L
             bo, bl = brute.decode_token(w.q_bits[b, i].tolist(), w.kv_bits.tolist(),
                                         w.block_table.tolist(), b, L, limit, SCALE)
+            np.testing.assert_allclose(out[b, i], np.array(bo), rtol=0, atol=1e-12)
+            np.testing.assert_allclose(lse[b, :, i], np.array(bl), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal,s_q,lens", [(False, 1, [100, 37]), (True, 2, [70, 3])])
+def test_oracle_matches_brute_force_fp8_dense(causal, s_q, lens):
+    h_q = 2
+    w = I.make_workload("brute8", len(lens), s_q, h_q, lens, causal=causal, fp8=True, seed=17 + s_q)
+    out, lse = O.decode(w.q_bits, w.block_table, w.cache_seqlens, kv_fp8=w.kv_fp8, causal=causal)
+    kv = w.kv_fp8.tolist()
+    for b, L in enumerate(lens):
+        for i in range(s_q):
+            limit = L - s_q + i + 1 if causal else L
+            bo, bl = brute.decode_token(w.q_bits[b, i].tolist(), None, w.block_table.tolist(), b, L, limit,
+                                        SCALE, kv_fp8=kv)
+            np.testing.assert_allclose(out[b, i], np.array(bo), rtol=0, atol=1e-12)
+            np.testing.assert_allclose(lse[b, :, i], np.array(bl), rtol=0, atol=1e-12)
+
+
+def test_oracle_matches_brute_force_sparse():
+    # padding, out-of-range positions and a duplicate in the index lists
+    w = I.make_workload("brutes", 2, 2, 2, [150, 90], fp8=True, topk=40, seed=19)
+    idx = w.indices.copy()
+    idx[0, 0, -5:] = -1
+    idx[0, 1, 3] = 150                   # == L: outside the sequence, skipped
+    idx[1, 0, 7] = idx[1, 0, 8]          # listed twice
+    idx[1, 1, :] = -1
+    idx[1, 1, 0] = 89
+    out, lse = O.decode(w.q_bits, w.block_table, w.cache_seqlens, kv_fp8=w.kv_fp8, indices=idx)
+    kv = w.kv_fp8.tolist()
+    for b, L in enumerate(w.cache_seqlens.tolist()):
+        for i in range(2):
+            bo, bl = brute.decode_token_sparse(w.q_bits[b, i].tolist(), kv, w.block_table.tolist(), b, L,
+                                               idx[b, i].tolist(), SCALE)
             np.testing.assert_allclose(out[b, i], np.array(bo), rtol=0, atol=1e-12)
             np.testing.assert_allclose(lse[b, :, i], np.array(bl), rtol=0, atol=1e-12)
 
@@ -200,7 +234,8 @@ def test_sparse_single_valid_index_and_all_padding():
     idx = np.full_like(w.indices, -1)
     idx[0, 0, 17] = 211
     o, l = O.decode(w.q_bits, w.block_table, w.cache_seqlens, kv_fp8=w.kv_fp8, indices=idx)
-    k = O.gather_rows(w.block_table, 0, np.array([211]), kv_fp8=w.kv_fp8)[0]
+    # the key straight from its stored row (page from the block table, slot 211 % 64)
+    k = fp8_rows_to_f64(w.kv_fp8[w.block_table[0, 211 // 64], 211 % 64, 0])
     q = bf16_bits_to_f64(w.q_bits[0, 0])
     np.testing.assert_array_equal(o[0, 0], np.broadcast_to(k[:512], o[0, 0].shape))
     np.testing.assert_allclose(l[0, :, 0], SCALE * (q @ k), rtol=0, atol=1e-12)

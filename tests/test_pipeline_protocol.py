@@ -1,7 +1,9 @@
-"""The decode kernel's barrier protocol, checked on a host-side model (CPU).
+"""The decode kernels' barrier protocols, checked on host-side models (CPU).
 
-`pipeline_model` restates the hand-offs of one CTA of the decode kernel:
-- the page producer: TMA, or 8 gather warps on the FP8 path;
+`pipeline_model` restates the hand-offs of one CTA of the bf16 decode kernel
+(and, in `Fp8Model`, of the FP8 kernel, with its two-pass QK^T and the V'
+rewrite by the gather warps):
+- the page producer: TMA, or 8 gather warps on the FP8 kernel;
 - the MMA warp's event loop;
 - four softmax warps, with padding warps, lazy rescales, segment epilogues and
   query-tile staging.
@@ -24,18 +26,38 @@ def _plan(rng, fp8, live=None, p_rescale=0.3):
     return PM.Plan(segs, live, fp8, resc)
 
 
-@pytest.mark.parametrize("fp8", [False, True])
-def test_protocol_runs_clean_on_random_schedules(fp8):
+def test_protocol_runs_clean_on_random_schedules():
     for seed in range(150):
         rng = random.Random(seed)
-        PM.Model(_plan(rng, fp8), seed).run()
+        PM.Model(_plan(rng, False), seed).run()
 
 
 def test_single_page_and_single_warp_edges():
     for seed in range(50):
         PM.Model(PM.Plan([1], 1, False, {}), seed).run()
-        PM.Model(PM.Plan([1, 1, 1, 1, 1], 4, True, {}), seed).run()
+        PM.Model(PM.Plan([1, 1, 1, 1, 1], 4, False, {}), seed).run()
         PM.Model(PM.Plan([7], 4, False, {(w, t): True for w in range(4) for t in range(7)}), seed).run()
+
+
+def test_fp8_protocol_runs_clean_on_random_schedules():
+    for seed in range(150):
+        rng = random.Random(seed)
+        PM.Fp8Model(_plan(rng, True), seed).run()
+    for seed in range(30):
+        PM.Fp8Model(PM.Plan([1], 1, True, {}), seed).run()
+        PM.Fp8Model(PM.Plan([1, 1, 1, 1, 1], 4, True, {}), seed).run()
+
+
+@pytest.mark.parametrize("mutation", ["no_sa_wait", "early_p", "early_v", "no_seg_end_pv"])
+def test_fp8_planted_mistakes_are_caught(mutation):
+    caught = 0
+    for seed in range(60):
+        rng = random.Random(seed)
+        try:
+            PM.Fp8Model(_plan(rng, True, live=PM.WARPS, p_rescale=0.5), seed, mutation=mutation).run()
+        except PM.ProtocolError:
+            caught += 1
+    assert caught > 0
 
 
 @pytest.mark.parametrize("mutation", ["shared_p_full", "no_rescale_wait", "single_pv_barrier"])

@@ -53,6 +53,8 @@ CASES = {
     "bf16 h64 causal s_q=2": lambda: RC.bf16_case(64, 2, True),
     "fp8 dense": RC.fp8_dense_case,
     "fp8 sparse": RC.fp8_sparse_case,
+    "fp8 dense x17 scales": lambda: RC.fp8_dense_case(x17=True),
+    "fp8 sparse x17 scales": lambda: RC.fp8_sparse_case(x17=True),
 }
 
 
@@ -60,6 +62,18 @@ CASES = {
 def test_rescale_cases_move_the_running_max(name):
     w = CASES[name]()
     assert _jumping_rows(w, 0) > 0
+
+
+@pytest.mark.parametrize("name", ["fp8 dense x17 scales", "fp8 sparse x17 scales"])
+def test_x17_cases_reach_large_logits(name):
+    # the boosted rows give natural-log logits of 30 or more, where a 2^-11
+    # relative rounding of a key value would move the lse by ~1e-3 or more
+    w = CASES[name]()
+    q = bf16_bits_to_f64(w.q_bits[0])
+    L = int(w.cache_seqlens[0])
+    keys = gather_rows(w.block_table, 0, np.arange(L), kv_fp8=w.kv_fp8)
+    s = (q[0] @ keys.T) * w.softmax_scale
+    assert s.max() >= 30.0
 
 
 def test_unboosted_workloads_do_not():

@@ -11,6 +11,7 @@ This file is collected last on purpose: if it fails, a run that stops at the
 first failure has already run every other test.
 """
 import ctypes
+import gc
 
 import numpy as np
 import pytest
@@ -64,18 +65,26 @@ def test_noalloc_matches_mla_decode_on_two_calls():
 
 def test_noalloc_allocates_nothing():
     w = I.make_config(2, batch=8, seqlen=1000)
-    _, call = _calls(w)
+    ref, call = _calls(w)                                                 # both stay alive throughout
     call.decode_noalloc()                                                 # warm-up: module and symbol set up
     torch.cuda.synchronize()
-    torch_before = torch.cuda.memory_allocated()
-    free_before, _ = torch.cuda.mem_get_info()
-    for _ in range(3):
-        call.decode_noalloc()
-    torch.cuda.synchronize()
-    free_after, _ = torch.cuda.mem_get_info()
-    assert torch.cuda.memory_allocated() == torch_before
+    # no Python garbage collection may free other tests' tensors in between
+    gc.collect()
+    gc.disable()
+    try:
+        torch_before = torch.cuda.memory_allocated()
+        free_before, _ = torch.cuda.mem_get_info()
+        for i in range(3):
+            call.decode_noalloc()
+        torch.cuda.synchronize()
+        free_after, total = torch.cuda.mem_get_info()
+        torch_after = torch.cuda.memory_allocated()
+    finally:
+        gc.enable()
+    assert torch_after == torch_before
     assert free_after == free_before
     assert int(call._keep[9].item()) == 0
+    del ref
 
 
 def test_noalloc_rejects_plans_beyond_its_scratch():
