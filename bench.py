@@ -524,26 +524,39 @@ def main():
     t, stream, flush = tm.t, tm.stream, tm.flush
 
     # ---- end to end through the public API, host buffers, copies in the region
-    q_host = t["q"].cpu().pin_memory()
-    bt_host = t["bt"].cpu().pin_memory()
-    sl_host = t["sl"].cpu().pin_memory()
-    idx_host = t["idx"].cpu().pin_memory() if t["idx"] is not None else None
+    # A step's inputs (q, block_table, cache_seqlens and the sparse indices)
+    # sit in one pinned host buffer and travel in one copy, as a serving
+    # engine would stage them; the device side is a buffer of the same
+    # layout, viewed as the four tensors.
+    parts = [("q", t["q"]), ("bt", t["bt"]), ("sl", t["sl"])] + ([("idx", t["idx"])] if t["idx"] is not None else [])
+    offs, in_bytes = {}, 0
+    for name, x in parts:
+        offs[name] = in_bytes
+        in_bytes += (x.numel() * x.element_size() + 255) // 256 * 256
+    in_host = torch.empty((in_bytes,), dtype=torch.uint8).pin_memory()
+    for name, x in parts:
+        nb = x.numel() * x.element_size()
+        in_host[offs[name]:offs[name] + nb].copy_(x.cpu().contiguous().view(-1).view(torch.uint8))
+
+    def device_inputs():
+        buf = torch.empty((in_bytes,), dtype=torch.uint8, device=dev)
+        views = {name: buf[offs[name]:offs[name] + x.numel() * x.element_size()].view(x.dtype).view(x.shape)
+                 for name, x in parts}
+        views["buf"] = buf
+        views.setdefault("idx", None)
+        return views
+
     out_host = torch.empty((w.batch, w.s_q, w.h_q, 512), dtype=torch.bfloat16).pin_memory()
     lse_host = torch.empty((w.batch, w.h_q, w.s_q), dtype=torch.float32).pin_memory()
-    q_dev, bt_dev, sl_dev = torch.empty_like(t["q"]), torch.empty_like(t["bt"]), torch.empty_like(t["sl"])
-    idx_dev = torch.empty_like(t["idx"]) if t["idx"] is not None else None
-    h2d = q_host.numel() * 2 + bt_host.numel() * 4 + sl_host.numel() * 4 + (idx_host.numel() * 4 if idx_host is not None else 0)
+    h2d = in_bytes
     d2h = out_host.numel() * 2 + lse_host.numel() * 4
+    din = device_inputs()
 
     def e2e_step():
-        q_dev.copy_(q_host, non_blocking=True)
-        bt_dev.copy_(bt_host, non_blocking=True)
-        sl_dev.copy_(sl_host, non_blocking=True)
-        if idx_dev is not None:
-            idx_dev.copy_(idx_host, non_blocking=True)
-        md_, ns_ = M.get_mla_metadata(sl_dev, w.s_q * w.h_q, 1, s_q=w.s_q, topk=w.topk if w.fp8 else None)
-        o, l = M.flash_mla_with_kvcache(q_dev, t["kv"], bt_dev, sl_dev, 512, md_, ns_, w.softmax_scale, w.causal,
-                                        w.fp8, idx_dev)
+        din["buf"].copy_(in_host, non_blocking=True)
+        md_, ns_ = M.get_mla_metadata(din["sl"], w.s_q * w.h_q, 1, s_q=w.s_q, topk=w.topk if w.fp8 else None)
+        o, l = M.flash_mla_with_kvcache(din["q"], t["kv"], din["bt"], din["sl"], 512, md_, ns_, w.softmax_scale,
+                                        w.causal, w.fp8, din["idx"])
         out_host.copy_(o, non_blocking=True)
         lse_host.copy_(l, non_blocking=True)
 
@@ -575,11 +588,10 @@ def main():
         cin, cout = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         sets = []
         for _ in range(2):
-            sets.append({
-                "q": torch.empty_like(t["q"]), "bt": torch.empty_like(t["bt"]), "sl": torch.empty_like(t["sl"]),
-                "idx": torch.empty_like(t["idx"]) if t["idx"] is not None else None,
-                "out": torch.empty_like(out_host).pin_memory(), "lse": torch.empty_like(lse_host).pin_memory(),
-                "ready": torch.cuda.Event(), "done": torch.cuda.Event()})
+            S = device_inputs()
+            S.update({"out": torch.empty_like(out_host).pin_memory(), "lse": torch.empty_like(lse_host).pin_memory(),
+                      "ready": torch.cuda.Event(), "done": torch.cuda.Event()})
+            sets.append(S)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         a.record(stream)
@@ -589,11 +601,7 @@ def main():
             with torch.cuda.stream(cin):
                 if k >= 2:
                     cin.wait_event(S["done"])          # step k-2 has finished reading this set
-                S["q"].copy_(q_host, non_blocking=True)
-                S["bt"].copy_(bt_host, non_blocking=True)
-                S["sl"].copy_(sl_host, non_blocking=True)
-                if S["idx"] is not None:
-                    S["idx"].copy_(idx_host, non_blocking=True)
+                S["buf"].copy_(in_host, non_blocking=True)
                 S["ready"].record(cin)
             stream.wait_event(S["ready"])
             md_, ns_ = M.get_mla_metadata(S["sl"], w.s_q * w.h_q, 1, s_q=w.s_q, topk=w.topk if w.fp8 else None)
@@ -654,7 +662,7 @@ def main():
         head_rec["cpu_baseline"] = line.get("cpu_baseline")
         head_rec["steps"] = args.steps
         head_rec["gpu_launches"] = 3 * args.steps
-        del q_dev, bt_dev, sl_dev, idx_dev, t, tm
+        din = sets = t = tm = None   # release the headline workload's device buffers
         torch.cuda.empty_cache()
         for key in PER_CONFIG:
             if key == head_key:

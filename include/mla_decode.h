@@ -222,6 +222,24 @@ MLA_API int mla_fp8_cache_write(const void* k_new, int64_t k_row_stride, int32_t
                                 void* kv_cache, int64_t k_block_stride, int32_t num_blocks, int32_t* err_word,
                                 void* stream);
 
+/*
+ * Give-up limit, in nanoseconds, of the decode kernels' pipeline waits for
+ * every decode call launched after this one (0 restores the default of 2 s).
+ * A wait that runs past it makes its CTA raise MLA_DEVERR_TIMEOUT in
+ * *err_word, drain its own copies and MMAs (those drains always keep the 2 s
+ * bound), free its tensor memory and return; the call's out/lse are then
+ * undefined, and the next call with the default limit computes normally.
+ * This exists to exercise that failure path: the bounded waits are the
+ * library's failure detection (a stuck pipeline ends the kernel with an
+ * error bit instead of hanging the GPU), and a short limit makes them give
+ * up on ordinary inputs.  Limits below 1 ms make the waits poll without
+ * suspending the waiting thread (slower, but each test is short enough to
+ * see such a limit pass).  It is process-wide and not meant to change while
+ * calls from other threads are being launched.  The pages have no
+ * counterpart to it.  Returns MLA_OK.
+ */
+MLA_API int mla_set_pipeline_wait_limit(uint64_t ns);
+
 /* Human-readable name of a status code (static string). */
 MLA_API const char* mla_status_string(int status);
 

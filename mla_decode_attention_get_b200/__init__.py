@@ -30,8 +30,24 @@ __all__ = ["get_mla_metadata", "flash_mla_with_kvcache", "MlaError", "mla_get_me
            "mla_workspace_bytes", "DecodeCall", "fp8_cache_write"]
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream_ptr(device) -> int:
+    """Handle of the current CUDA stream of ``device`` (a torch.device)."""
+    if _raw_stream is not None:
+        idx = device.index
+        return _raw_stream(torch.cuda.current_device() if idx is None else idx)
     return torch.cuda.current_stream(device).cuda_stream
+
+
+# Host-side plan sizes are pure functions of the shapes (and of the device's
+# SM count): cache them, so that a decode step costs no extra library calls.
+_shape_cache = {}
+_ws_cache = {}
+# Error word of calls made with check=False: nobody reads it, so all such
+# calls on a device share one (the kernels only OR bits into it).
+_discard_err = {}
 
 
 def _require(cond: bool, msg: str) -> None:
@@ -49,6 +65,33 @@ def mla_metadata_shape(batch: int, s_q: int, h_q: int, h_kv: int = 1, topk: int 
 
 def mla_workspace_bytes(batch: int, s_q: int, h_q: int, topk: int, num_parts: int) -> int:
     return _abi.workspace_bytes(batch, s_q, h_q, topk, num_parts)
+
+
+def _metadata_shape_of(batch, s_q, h_q, h_kv, topk, num_sm_parts, device) -> Tuple[int, int]:
+    key = (batch, s_q, h_q, h_kv, topk, num_sm_parts, device.index)
+    r = _shape_cache.get(key)
+    if r is None:
+        with torch.cuda.device(device):
+            r = mla_metadata_shape(batch, s_q, h_q, h_kv, topk, num_sm_parts)
+        _shape_cache[key] = r
+    return r
+
+
+def _workspace_bytes_of(batch, s_q, h_q, topk, num_parts) -> int:
+    key = (batch, s_q, h_q, topk, num_parts)
+    r = _ws_cache.get(key)
+    if r is None:
+        r = mla_workspace_bytes(batch, s_q, h_q, topk, num_parts)
+        _ws_cache[key] = r
+    return r
+
+
+def _discard_err_word(device) -> torch.Tensor:
+    e = _discard_err.get(device.index)
+    if e is None:
+        e = torch.zeros((1,), dtype=torch.int32, device=device)
+        _discard_err[device.index] = e
+    return e
 
 
 def mla_get_metadata(cache_seqlens: torch.Tensor, batch: int, s_q: int, h_q: int, h_kv: int, topk: int,
@@ -146,17 +189,55 @@ def get_mla_metadata(cache_seqlens: torch.Tensor, num_q_tokens_per_head_k: int, 
     ``cache_seqlens``."""
     _require(cache_seqlens.is_cuda and cache_seqlens.dtype == torch.int32 and cache_seqlens.dim() == 1,
              "cache_seqlens must be a 1-D int32 CUDA tensor")
-    cache_seqlens = cache_seqlens.contiguous()
+    if cache_seqlens.stride(0) != 1:
+        cache_seqlens = cache_seqlens.contiguous()
     batch = cache_seqlens.shape[0]
     rows = num_q_tokens_per_head_k * num_heads_k
     _require(rows % s_q == 0, "s_q must divide s_q*h_q")
     h_q = rows // s_q
     tk = int(topk or 0)
-    parts, nlen = mla_metadata_shape(batch, s_q, h_q, num_heads_k, tk, int(num_sm_parts or 0))
-    tile_md = torch.empty((parts, _abi.MD_WORDS), dtype=torch.int32, device=cache_seqlens.device)
-    num_splits = torch.empty((nlen,), dtype=torch.int32, device=cache_seqlens.device)
-    mla_get_metadata(cache_seqlens, batch, s_q, h_q, num_heads_k, tk, tile_md, num_splits)
+    dev = cache_seqlens.device
+    parts, nlen = _metadata_shape_of(batch, s_q, h_q, num_heads_k, tk, int(num_sm_parts or 0), dev)
+    # one allocation: tile_md [parts, 8] then num_splits [nlen]
+    buf = torch.empty((parts * _abi.MD_WORDS + nlen,), dtype=torch.int32, device=dev)
+    tile_md = buf[:parts * _abi.MD_WORDS].view(parts, _abi.MD_WORDS)
+    num_splits = buf[parts * _abi.MD_WORDS:]
+    _abi.check(_abi.lib().mla_get_metadata(
+        cache_seqlens.data_ptr(), batch, s_q, h_q, num_heads_k, tk, parts, tile_md.data_ptr(),
+        num_splits.data_ptr(), _stream_ptr(dev)), "mla_get_metadata")
     return tile_md, num_splits
+
+
+def _check_decode_inputs(q, k_cache, block_table, cache_seqlens, head_dim_v, is_fp8_kvcache, indices):
+    """Validate the decode inputs (host checks only); returns the cache as
+    the library reads it (the FP8 cache viewed as bytes)."""
+    _require(q.is_cuda and q.dtype == torch.bfloat16 and q.dim() == 4 and q.shape[-1] == D_QK,
+             "q must be bf16 [batch, s_q, h_q, 576] on CUDA")
+    b, s_q, h_q, _ = q.shape
+    qs = q.stride()
+    _require(qs[3] == 1 and (h_q == 1 or qs[2] == D_QK) and (s_q == 1 or qs[1] == h_q * D_QK),
+             "q must be contiguous within a batch entry")
+    _require(head_dim_v == D_V, "head_dim_v must be 512")
+    _require(k_cache.dim() == 4 and k_cache.shape[1] == PAGE_SIZE, "k_cache must be [blocks, 64, h_kv, d]")
+    if is_fp8_kvcache:
+        if k_cache.dtype != torch.uint8:
+            k_cache = k_cache.view(torch.uint8)
+        _require(k_cache.shape[-1] == FP8_ROW_BYTES, "fp8 cache rows must be 656 bytes")
+    else:
+        _require(k_cache.dtype == torch.bfloat16 and k_cache.shape[-1] == D_QK, "bf16 cache rows must be 576 wide")
+    ks = k_cache.stride()
+    d = k_cache.shape[3]
+    _require(ks[3] == 1 and (k_cache.shape[2] == 1 or ks[2] == d) and ks[1] == k_cache.shape[2] * d,
+             "each cache page must be contiguous")
+    _require(block_table.dtype == torch.int32 and block_table.dim() == 2 and block_table.stride(1) == 1,
+             "block_table must be int32 [batch, max_blocks] with unit column stride")
+    _require(cache_seqlens.dtype == torch.int32 and cache_seqlens.dim() == 1 and cache_seqlens.stride(0) == 1,
+             "cache_seqlens must be contiguous int32")
+    if indices is not None:
+        _require(is_fp8_kvcache, "sparse indices are read with the fp8 cache only")
+        _require(indices.dtype == torch.int32 and indices.dim() == 3 and indices.shape[:2] == (b, s_q)
+                 and indices.is_contiguous(), "indices must be contiguous int32 [batch, s_q, topk]")
+    return k_cache
 
 
 def prepare_decode(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.Tensor,
@@ -165,38 +246,19 @@ def prepare_decode(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.Te
                    is_fp8_kvcache: bool = False, indices: Optional[torch.Tensor] = None) -> DecodeCall:
     """Validate shapes, allocate out / lse / workspace / error word, and
     marshal one decode call."""
-    _require(q.is_cuda and q.dtype == torch.bfloat16 and q.dim() == 4 and q.shape[-1] == D_QK,
-             "q must be bf16 [batch, s_q, h_q, 576] on CUDA")
-    _require(q[0].is_contiguous(), "q must be contiguous within a batch entry")
-    _require(head_dim_v == D_V, "head_dim_v must be 512")
-    _require(k_cache.dim() == 4 and k_cache.shape[1] == PAGE_SIZE, "k_cache must be [blocks, 64, h_kv, d]")
-    h_kv = k_cache.shape[2]
-    if is_fp8_kvcache:
-        if k_cache.dtype != torch.uint8:
-            k_cache = k_cache.view(torch.uint8)
-        _require(k_cache.shape[-1] == FP8_ROW_BYTES, "fp8 cache rows must be 656 bytes")
-    else:
-        _require(k_cache.dtype == torch.bfloat16 and k_cache.shape[-1] == D_QK, "bf16 cache rows must be 576 wide")
-    _require(k_cache[0].is_contiguous(), "each cache page must be contiguous")
-    _require(block_table.dtype == torch.int32 and block_table.dim() == 2 and block_table.stride(1) == 1,
-             "block_table must be int32 [batch, max_blocks] with unit column stride")
-    _require(cache_seqlens.dtype == torch.int32 and cache_seqlens.is_contiguous(), "cache_seqlens must be int32")
+    k_cache = _check_decode_inputs(q, k_cache, block_table, cache_seqlens, head_dim_v, is_fp8_kvcache, indices)
     b, s_q, h_q, _ = q.shape
-    if indices is not None:
-        _require(is_fp8_kvcache, "sparse indices are read with the fp8 cache only")
-        _require(indices.dtype == torch.int32 and indices.dim() == 3 and indices.shape[:2] == (b, s_q)
-                 and indices.is_contiguous(), "indices must be contiguous int32 [batch, s_q, topk]")
     topk = indices.shape[-1] if indices is not None else 0
     if softmax_scale is None:
         softmax_scale = D_QK ** -0.5
     dev = q.device
     out = torch.empty((b, s_q, h_q, D_V), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=dev)
-    ws = torch.empty((mla_workspace_bytes(b, s_q, h_q, topk, tile_scheduler_metadata.shape[0]),),
+    ws = torch.empty((_workspace_bytes_of(b, s_q, h_q, topk, tile_scheduler_metadata.shape[0]),),
                      dtype=torch.uint8, device=dev)
     err = torch.zeros((1,), dtype=torch.int32, device=dev)
     return DecodeCall(q, k_cache, block_table, cache_seqlens, tile_scheduler_metadata, num_splits, out, lse,
-                      ws, err, softmax_scale, causal, is_fp8_kvcache, indices, h_kv)
+                      ws, err, softmax_scale, causal, is_fp8_kvcache, indices, k_cache.shape[2])
 
 
 def flash_mla_with_kvcache(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.Tensor,
@@ -206,11 +268,27 @@ def flash_mla_with_kvcache(q: torch.Tensor, k_cache: torch.Tensor, block_table: 
                            check: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
     """MLA decode: returns (out bf16 [batch, s_q, h_q, 512], lse fp32
     [batch, h_q, s_q]).  With ``check=True`` the call synchronises and raises
-    if a kernel reported a data error (bad block_table entry or index)."""
-    call = prepare_decode(q, k_cache, block_table, cache_seqlens, head_dim_v, tile_scheduler_metadata,
-                          num_splits, softmax_scale, causal, is_fp8_kvcache, indices)
-    call.decode()
-    out, lse, err = call._keep[6], call._keep[7], call._keep[9]
+    if a kernel reported a data error (bad block_table entry or index);
+    without it the error bits go to a word nobody reads."""
+    k_cache = _check_decode_inputs(q, k_cache, block_table, cache_seqlens, head_dim_v, is_fp8_kvcache, indices)
+    b, s_q, h_q, _ = q.shape
+    topk = indices.shape[-1] if indices is not None else 0
+    if softmax_scale is None:
+        softmax_scale = D_QK ** -0.5
+    dev = q.device
+    num_parts = tile_scheduler_metadata.shape[0]
+    out = torch.empty((b, s_q, h_q, D_V), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=dev)
+    ws_bytes = _workspace_bytes_of(b, s_q, h_q, topk, num_parts)
+    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    err = torch.zeros((1,), dtype=torch.int32, device=dev) if check else _discard_err_word(dev)
+    a = _abi.DecodeArgs(q.data_ptr(), q.stride(0), k_cache.data_ptr(), k_cache.stride(0) * k_cache.element_size(),
+                        k_cache.shape[0], block_table.data_ptr(), block_table.stride(0), block_table.shape[1],
+                        cache_seqlens.data_ptr(), indices.data_ptr() if indices is not None else None, topk,
+                        tile_scheduler_metadata.data_ptr(), num_splits.data_ptr(), num_parts, out.data_ptr(),
+                        lse.data_ptr(), ws.data_ptr(), ws_bytes, err.data_ptr(), b, s_q, h_q, k_cache.shape[2],
+                        D_V, float(softmax_scale), 1 if causal else 0, 1 if is_fp8_kvcache else 0)
+    _abi.check(_abi.lib().mla_decode(ctypes.byref(a), _stream_ptr(dev)), "mla_decode")
     if check:
         e = int(err.item())
         if e:

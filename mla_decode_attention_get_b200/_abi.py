@@ -31,7 +31,7 @@ FP8_ROW_BYTES = 656
 # Every symbol include/mla_decode.h declares.
 EXPORTS = ("mla_metadata_shape", "mla_get_metadata", "mla_workspace_bytes", "mla_decode",
            "mla_decode_attention", "mla_decode_combine", "mla_decode_noalloc", "mla_fp8_cache_write",
-           "mla_status_string")
+           "mla_set_pipeline_wait_limit", "mla_status_string")
 
 # Size of the scratch array built into the library for mla_decode_noalloc.
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -93,6 +93,7 @@ def lib() -> ctypes.CDLL:
         for name in ("mla_decode", "mla_decode_attention", "mla_decode_combine", "mla_decode_noalloc"):
             getattr(L, name).argtypes = [p(DecodeArgs), v]
         L.mla_fp8_cache_write.argtypes = [v, ctypes.c_int64, i, v, v, ctypes.c_int64, i, v, v]
+        L.mla_set_pipeline_wait_limit.argtypes = [ctypes.c_uint64]
         L.mla_status_string.argtypes = [i]
         L.mla_status_string.restype = ctypes.c_char_p
         for name in EXPORTS[:-1]:
@@ -115,6 +116,12 @@ def metadata_shape(batch, s_q, h_q, h_kv, topk, num_sm_parts):
     check(lib().mla_metadata_shape(batch, s_q, h_q, h_kv, topk, num_sm_parts,
                                    ctypes.byref(parts), ctypes.byref(nlen)), "mla_metadata_shape")
     return parts.value, nlen.value
+
+
+def set_pipeline_wait_limit(ns: int) -> None:
+    """Give-up limit of the kernels' pipeline waits for the calls that follow
+    (0 = the default); see mla_set_pipeline_wait_limit."""
+    check(lib().mla_set_pipeline_wait_limit(int(ns)), "mla_set_pipeline_wait_limit")
 
 
 def workspace_bytes(batch, s_q, h_q, topk, num_parts) -> int:

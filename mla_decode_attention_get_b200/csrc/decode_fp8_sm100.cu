@@ -39,10 +39,11 @@
 //    bf16 RoPE); the RoPE chunk holds the tile's P (f16) once QK^T of the
 //    tile has completed.
 //  * TMEM (M = 64 layout: 16 lanes of each 32-lane quadrant): O in lanes
-//    0-15 (512 columns); lanes 16-31 hold three partial-S buffers (columns
-//    0-191), the query's latent dims (192-447) and its RoPE dims (448-479).
-//    QK^T runs in two passes per tile: groups 0-2 into buffers 0-2, then
-//    group 3 and RoPE into buffers 0-1 once the softmax has read them.
+//    0-15 (512 columns); lanes 16-31 hold a ring of three partial-S slots
+//    (columns 0-191), the query's latent dims (192-447) and its RoPE dims
+//    (448-479).  QK^T of a tile is five parts (latent groups 0-3, RoPE), each
+//    into the next slot once the softmax has read the slot's previous part,
+//    so the MMAs of one tile overlap the softmax of the one before.
 //  * Every wait is bounded; on timeout the CTA raises MLA_DEVERR_TIMEOUT,
 //    drains its own MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
@@ -60,6 +61,22 @@ namespace mla {
 // hand-offs of every tile in the first kFp8TraceCtas CTAs of row tile 0.
 constexpr int kFp8TraceCtas = 4, kFp8TraceEvents = 16, kFp8TraceTiles = 256;
 __device__ unsigned long long g_fp8_trace[kFp8TraceCtas][kFp8TraceEvents][kFp8TraceTiles];
+// Per CTA (all of them): %globaltimer at entry, after the set-up and the
+// dependency wait, and at exit, and the SM it ran on.
+constexpr int kFp8SpanCtas = 1024;
+__device__ unsigned long long g_fp8_span[kFp8SpanCtas][4];
+#define FP8_SPAN(k)                                                              \
+  do {                                                                           \
+    const unsigned cta = blockIdx.y * gridDim.x + blockIdx.x;                    \
+    if (threadIdx.x == 0 && cta < kFp8SpanCtas) {                                \
+      g_fp8_span[cta][k] = globaltimer_ns();                                     \
+      if ((k) == 0) {                                                            \
+        unsigned sm;                                                             \
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));                          \
+        g_fp8_span[cta][3] = sm;                                                 \
+      }                                                                          \
+    }                                                                            \
+  } while (0)
 #define FP8_TRACE(ev, idx)                                                                      \
   do {                                                                                          \
     if (blockIdx.x < kFp8TraceCtas && blockIdx.y == 0 && (idx) >= 0 && (idx) < kFp8TraceTiles)  \
@@ -68,6 +85,9 @@ __device__ unsigned long long g_fp8_trace[kFp8TraceCtas][kFp8TraceEvents][kFp8Tr
 #else
 #define FP8_TRACE(ev, idx) \
   do {                     \
+  } while (0)
+#define FP8_SPAN(k) \
+  do {              \
   } while (0)
 #endif
 
@@ -82,10 +102,13 @@ constexpr uint32_t kColQ = 192;                // query latent dims (f16 pairs),
 constexpr uint32_t kColQRope = 448;            // query RoPE dims (bf16 pairs), lanes 16-31
 constexpr int kRopeChunk = kChunks - 1;        // chunk 8: RoPE; then P of the tile
 constexpr int kStageBytes = kPageBytes;        // 73728
-// The four scales of key k of a stage sit at float4 k + k / 32 of the
-// stage's scale block: keys k and k + 32 (read together by the two halves of
-// a softmax warp) then fall in different banks.
-constexpr int kScaleStride = kPage + 2;        // float4 per stage
+// The scales of a stage: [group][key] fp32, so that a softmax thread reads the
+// group-g scales of its 32 keys as eight 16-byte loads.
+constexpr int kScaleFloats = 4 * kPage;        // per stage
+// QK^T of a tile is five parts (latent groups 0-3, then RoPE), each written
+// into the next slot of a ring of partial-S buffers in TMEM.
+constexpr int kParts = 5;
+constexpr int kSlots = 3;
 constexpr int kRescaleGroupLog2 = 7;           // raise E_g once a scale reaches 2^(E_g + 7)
 
 constexpr int kWarpQPrefetch = 0, kWarpMma = 1, kWarpSoftmax0 = 2, kWarpGather0 = 6;
@@ -100,12 +123,12 @@ struct StageInfo {
 
 struct Smem {
   static constexpr int stage_off = 0;
-  static constexpr int scales_off = stage_off + kStages * kStageBytes;      // [stage][kScaleStride] float4
-  static constexpr int info_off = scales_off + kStages * kScaleStride * 16;
+  static constexpr int scales_off = stage_off + kStages * kStageBytes;      // [stage][group][key] float
+  static constexpr int info_off = scales_off + kStages * kScaleFloats * 4;
   static constexpr int bar_off = (info_off + kStages * static_cast<int>(sizeof(StageInfo)) + 7) & ~7;
-  // kv_full, kv_empty, p_full, qk_done, v_ready (per stage), sa_full, sa_empty, sb_full, sb_empty,
+  // kv_full, kv_empty, p_full, qk_done, v_ready (per stage), slot_full, slot_empty (per slot),
   // q_full, done
-  static constexpr int n_bars = 5 * kStages + 6;
+  static constexpr int n_bars = 5 * kStages + 2 * kSlots + 2;
   static constexpr int misc_off = bar_off + n_bars * 8;                     // tmem base, abort flag
   static constexpr int total = misc_off + 16;
   static_assert(kStageBytes % 1024 == 0 && kChunkBytes % 1024 == 0, "tiles must stay 1024-B aligned");
@@ -118,10 +141,8 @@ struct Bars {
   uint64_t* p_full;     // [stage] P of the stage's tile written (4 softmax warps)
   uint64_t* qk_done;    // [stage] both QK^T passes of the stage's tile completed (commit)
   uint64_t* v_ready;    // [stage] V' of the stage's tile written (8 gather warps)
-  uint64_t* sa_full;    // pass A (groups 0-2) of QK^T completed (commit)
-  uint64_t* sa_empty;   // pass A buffers read (4 softmax warps)
-  uint64_t* sb_full;    // pass B (group 3, RoPE) completed (commit)
-  uint64_t* sb_empty;   // pass B buffers read (4 softmax warps)
+  uint64_t* slot_full;  // [slot] a part of QK^T completed into the slot (commit)
+  uint64_t* slot_empty; // [slot] the slot was read (4 softmax warps)
   uint64_t* q_full;     // query tile of the next segment in TMEM (4 softmax warps)
   uint64_t* done;
 };
@@ -132,7 +153,20 @@ __device__ __forceinline__ int tile_valid_rows(const DecodeParams& p) {
 
 __device__ __forceinline__ uint8_t* stage_ptr(uint8_t* smem, int s) { return smem + Smem::stage_off + s * kStageBytes; }
 
-__device__ __forceinline__ int scale_index(int s, int k) { return s * kScaleStride + k + (k >> 5); }
+__device__ __forceinline__ int scale_index(int s, int g, int k) { return (s * 4 + g) * kPage + k; }
+
+// Position in the ring of partial-S slots; the MMA warp and the softmax warps
+// step through it in the same order (five parts per tile).
+struct Ring {
+  int slot = 0;
+  uint32_t phase = 0;
+  __device__ __forceinline__ void next() {
+    if (++slot == kSlots) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+};
 
 // 2^n for n in [-126, 127] (a normal fp32 number).
 __device__ __forceinline__ float pow2i(int n) { return __int_as_float((127 + n) << 23); }
@@ -180,15 +214,19 @@ struct GroupExp {
     return beta;
   }
 
-  // Update from a tile (its gather warps' per-group maxima); beta_g =
-  // 2^(E_old - E_new).  Returns whether some E_g moved.
-  __device__ __forceinline__ bool update(const StageInfo& si, float4& beta) {
+  // The tile's largest |scale| per group, from its gather warps' maxima.
+  __device__ __forceinline__ static float4 tile_max(const StageInfo& si) {
     float4 m = si.gmax[0];
 #pragma unroll
     for (int w = 1; w < kGatherWarps; ++w) {
       const float4 x = si.gmax[w];
       m = make_float4(fmaxf(m.x, x.x), fmaxf(m.y, x.y), fmaxf(m.z, x.z), fmaxf(m.w, x.w));
     }
+    return m;
+  }
+  // Update from a tile's per-group maxima; beta_g = 2^(E_old - E_new).
+  // Returns whether some E_g moved.
+  __device__ __forceinline__ bool update(const float4 m, float4& beta) {
     beta.x = step(e0, 0, m.x);
     beta.y = step(e1, 1, m.y);
     beta.z = step(e2, 2, m.z);
@@ -280,16 +318,16 @@ __device__ __forceinline__ void gather_role(const DecodeParams& p, const Partiti
   gexp.reset();
   auto rewrite = [&]() -> bool {
     const int s = tr % kStages;
-    if (!mbar_wait(&bars.qk_done[s], (tr / kStages) & 1, abort_flag)) return false;
+    if (!mbar_wait(&bars.qk_done[s], (tr / kStages) & 1, abort_flag, p.wait_ns)) return false;
     if (rwc.seg != rw_seg) {
       gexp.reset();
       rw_seg = rwc.seg;
     }
     float4 beta;
-    gexp.update(info[s], beta);
+    gexp.update(GroupExp::tile_max(info[s]), beta);
     const int e = lane >> 2, qq = lane & 3;
     const int k = 8 * gw + e;
-    const float sk = scales[4 * scale_index(s, k) + qq];
+    const float sk = scales[scale_index(s, qq, k)];
     const float f32 = sk * pow2i(-gexp.e(qq));
     const uint32_t f = pack_f16x2(f32, f32);
     uint8_t* row = stage_ptr(smem, s) + k * 128;
@@ -363,7 +401,7 @@ __device__ __forceinline__ void gather_role(const DecodeParams& p, const Partiti
         }
       }
       if (lane == 0 && gw == 0) FP8_TRACE(0, t);
-      if (!mbar_wait(&bars.kv_empty[s], ((t / kStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&bars.kv_empty[s], ((t / kStages) & 1) ^ 1, abort_flag, p.wait_ns)) { ok = false; break; }
       if (lane == 0 && gw == 0) FP8_TRACE(1, t);
       uint8_t* stage = stage_ptr(smem, s);
 #pragma unroll
@@ -395,9 +433,8 @@ __device__ __forceinline__ void gather_role(const DecodeParams& p, const Partiti
         }
         // the key's four scales: lane 0 holds groups 0 and 2, lane 16 groups 1 and 3
         if ((lane & 15) == 0) {
-          float* sk = scales + 4 * scale_index(s, k);
-          sk[lane >> 4] = s0[e];
-          sk[2 + (lane >> 4)] = s1[e];
+          scales[scale_index(s, lane >> 4, k)] = s0[e];
+          scales[scale_index(s, 2 + (lane >> 4), k)] = s1[e];
         }
         gm0 = fmaxf(gm0, fabsf(s0[e]));
         gm1 = fmaxf(gm1, fabsf(s1[e]));
@@ -442,15 +479,16 @@ __device__ __forceinline__ int stage_nvalid(const StageInfo& si) {
 // ---------------------------------------------------------------------------
 // Warp 1 (whole warp, one elected lane issues): the MMAs, in a fixed order per
 // tile t, each step after a (bounded, sleeping) wait for its inputs:
-//   pass A of QK^T(t)  (groups 0-2 into buffers 0-2): tile in, query tile in,
-//                      softmax done with pass B of t-1;
-//   pass B of QK^T(t)  (group 3 into buffer 0, RoPE into buffer 1): softmax
-//                      done with pass A of t;
-//   PV(t-1)            P and V' of t-1 written (they are by then: the softmax
-//                      wrote P(t-1) before reading pass A of t);
-//   PV(t)              only at the end of a segment, whose epilogue waits on it.
-// The tensor pipe runs PV(t-1) while the softmax reads pass B of t and QK^T
-// of t+1 while it finishes tile t.
+//   QK^T(t), five parts   latent groups 0-3 (8 MMAs each, f16 codes) and RoPE
+//                         (4 MMAs, bf16), each into the next slot of the
+//                         three-slot ring once the softmax has read the
+//                         slot's previous part; the first part also waits for
+//                         the tile and (at a segment start) the query tile;
+//   PV(t-1)               P and V' of t-1 written;
+//   PV(t)                 only at the end of a segment, whose epilogue waits
+//                         on it.
+// So the first three parts of tile t run while the softmax finishes tile t-1,
+// and PV(t-1) while it reads the parts of tile t.
 __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition& part, uint8_t* smem, Bars bars,
                                          uint32_t tmem_base, volatile int* abort_flag) {
   constexpr uint32_t idesc_qk = idesc_f16_f32(kRows, kPage, false, false);
@@ -458,10 +496,10 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
   constexpr uint32_t idesc_pv = idesc_f16_f32(kRows, 256, false, true);
   const StageInfo* info = reinterpret_cast<const StageInfo*>(smem + Smem::info_off);
   const uint32_t tmem_hi = tmem_base + (16u << 16);      // lanes 16-31 of each quadrant
-  const uint32_t ring = smem_u32(smem + Smem::stage_off);
-  const uint64_t k_desc0 = sdesc_sw128(ring, 16, 1024);
-  const uint64_t v_desc0 = sdesc_sw128(ring, kChunkBytes, 1024);
-  const uint64_t p_desc0 = sdesc_sw128(ring + kRopeChunk * kChunkBytes, 16, 1024);
+  const uint32_t ring_base = smem_u32(smem + Smem::stage_off);
+  const uint64_t k_desc0 = sdesc_sw128(ring_base, 16, 1024);
+  const uint64_t v_desc0 = sdesc_sw128(ring_base, kChunkBytes, 1024);
+  const uint64_t p_desc0 = sdesc_sw128(ring_base + kRopeChunk * kChunkBytes, 16, 1024);
 
   auto qk_chunk = [&](uint32_t d, uint64_t kd, uint32_t a_col, int c, uint32_t idesc, bool first_chunk) {
 #pragma unroll
@@ -473,8 +511,8 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
   int o_seg = -1;
   auto pv_tile = [&](int t, int seg, int nv) -> bool {
     const int s = t % kStages;
-    if (!mbar_wait(&bars.p_full[s], (t / kStages) & 1, abort_flag)) return false;
-    if (!mbar_wait(&bars.v_ready[s], (t / kStages) & 1, abort_flag)) return false;
+    if (!mbar_wait(&bars.p_full[s], (t / kStages) & 1, abort_flag, p.wait_ns)) return false;
+    if (!mbar_wait(&bars.v_ready[s], (t / kStages) & 1, abort_flag, p.wait_ns)) return false;
     tc_fence_after();
     FP8_TRACE(5, t);
     if (nv > 0) {
@@ -498,40 +536,41 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
   bool ok = true;
   bool have_prev = false;   // a tile whose PV is still to issue
   int prev_t = 0, prev_seg = 0, prev_nv = 0;
+  Ring ring;
   while (c.valid) {
     const int t = c.t;
     const int s = t % kStages;
     const bool first = (c.j == (c.u == part.u0 ? part.j0 : 0));
     const bool last = (c.j + 1 == c.je);
-    // pass A
-    if (!mbar_wait(&bars.kv_full[s], (t / kStages) & 1, abort_flag) ||
-        (first && !mbar_wait(bars.q_full, c.seg & 1, abort_flag)) ||
-        !mbar_wait(bars.sb_empty, (t & 1) ^ 1, abort_flag)) {
+    if (!mbar_wait(&bars.kv_full[s], (t / kStages) & 1, abort_flag, p.wait_ns) ||
+        (first && !mbar_wait(bars.q_full, c.seg & 1, abort_flag, p.wait_ns))) {
       ok = false;
       break;
     }
-    tc_fence_after();
-    FP8_TRACE(3, t);
     const int nv = stage_nvalid(info[s]);
     const uint64_t kd = k_desc0 + ((s * kStageBytes) >> 4);
-    if (nv > 0) {
-#pragma unroll
-      for (int g = 0; g < 3; ++g) {
-        qk_chunk(tmem_hi + 64 * g, kd, kColQ + 32 * (2 * g), 2 * g, idesc_qk, true);
-        qk_chunk(tmem_hi + 64 * g, kd, kColQ + 32 * (2 * g + 1), 2 * g + 1, idesc_qk, false);
+#pragma unroll 1
+    for (int i = 0; i < kParts; ++i) {
+      if (!mbar_wait(&bars.slot_empty[ring.slot], ring.phase ^ 1u, abort_flag, p.wait_ns)) {
+        ok = false;
+        break;
       }
+      tc_fence_after();
+      if (i == 0) FP8_TRACE(3, t);
+      if (i == kParts - 1) FP8_TRACE(4, t);
+      const uint32_t d = tmem_hi + 64 * ring.slot;
+      if (nv > 0) {
+        if (i < 4) {
+          qk_chunk(d, kd, kColQ + 32 * (2 * i), 2 * i, idesc_qk, true);
+          qk_chunk(d, kd, kColQ + 32 * (2 * i + 1), 2 * i + 1, idesc_qk, false);
+        } else {
+          qk_chunk(d, kd, kColQRope, kRopeChunk, idesc_rope, true);
+        }
+      }
+      umma_commit_elect(&bars.slot_full[ring.slot]);
+      ring.next();
     }
-    umma_commit_elect(bars.sa_full);
-    // pass B
-    if (!mbar_wait(bars.sa_empty, t & 1, abort_flag)) { ok = false; break; }
-    tc_fence_after();
-    FP8_TRACE(4, t);
-    if (nv > 0) {
-      qk_chunk(tmem_hi + 0, kd, kColQ + 32 * 6, 6, idesc_qk, true);
-      qk_chunk(tmem_hi + 0, kd, kColQ + 32 * 7, 7, idesc_qk, false);
-      qk_chunk(tmem_hi + 64, kd, kColQRope, kRopeChunk, idesc_rope, true);
-    }
-    umma_commit_elect(bars.sb_full);
+    if (!ok) break;
     umma_commit_elect(&bars.qk_done[s]);     // the codes may now become V'
     // PV of the previous tile, and of this one at the end of its segment
     if (have_prev && !pv_tile(prev_t, prev_seg, prev_nv)) { ok = false; break; }
@@ -651,6 +690,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
 
   int t = 0;
   bool ok = true;
+  Ring ring;
 
   for_each_segment(p, part, [&](int u, int jb, int je) -> bool {
     const UnitInfo ui = unit_info(p, u);
@@ -663,65 +703,74 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
     const int lim = ui.L - s_q + tok_dense + 1;      // causal: keys t < lim are visible
     for (int j = jb; j < je; ++j) {
       const int s = t % kStages;
-      if (!mbar_wait(&bars.kv_full[s], (t / kStages) & 1, abort_flag)) { ok = false; return false; }
-      if (!mbar_wait(bars.sa_full, t & 1, abort_flag)) { ok = false; return false; }
-      tc_fence_after();
-      if (lane == 0 && q4 == 2) FP8_TRACE(6, t);
+      if (!mbar_wait(&bars.kv_full[s], (t / kStages) & 1, abort_flag, p.wait_ns)) { ok = false; return false; }
+      // the tile's valid-key count, masks and per-group scale maxima, read
+      // while the first parts of QK^T run
       const int nv = stage_nvalid(info[s]);
       const bool work = nv > 0 && warp_live;
-      const float4* sck = reinterpret_cast<const float4*>(scales) + scale_index(s, key0);   // this half's keys
-      // pass A: groups 0-2
+      const uint32_t vmask = static_cast<uint32_t>(info[s].mask[4 * half]) |
+                             (static_cast<uint32_t>(info[s].mask[4 * half + 1]) << 8) |
+                             (static_cast<uint32_t>(info[s].mask[4 * half + 2]) << 16) |
+                             (static_cast<uint32_t>(info[s].mask[4 * half + 3]) << 24);
+      const float4 gmax = GroupExp::tile_max(info[s]);
+      const float* sck = scales + scale_index(s, 0, key0);   // group g of this half's keys: sck[g * kPage + i]
+      const float f = rho * scale_log2;
+      // the five parts of QK^T, each from its ring slot:
+      //   x = (sum_g scale[k][g] * S_g) * 2^e_r * scale_log2 + S_rope * scale_log2
       float x[32];
-      if (work) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) x[i] = 0.f;
+#pragma unroll 1
+      for (int i = 0; i < kParts; ++i) {
+        if (!mbar_wait(&bars.slot_full[ring.slot], ring.phase, abort_flag, p.wait_ns)) { ok = false; return false; }
+        tc_fence_after();
+        if (lane == 0 && q4 == 2 && i == 0) FP8_TRACE(6, t);
+        if (lane == 0 && q4 == 2 && i == kParts - 1) FP8_TRACE(8, t);
         float y[32];
-        tmem_ld_16x32bx2_x32(s_taddr + 0, x);
-        tmem_ld_16x32bx2_x32(s_taddr + 64, y);
+        if (work) tmem_ld_16x32bx2_x32(s_taddr + 64 * ring.slot, y);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.slot_empty[ring.slot]);
+        ring.next();
+        if (work) {
+          if (i < 4) {
+            const float4* sg = reinterpret_cast<const float4*>(sck + i * kPage);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float4 sc = sck[i];
-          x[i] = x[i] * sc.x + y[i] * sc.y;
+            for (int q = 0; q < 8; ++q) {
+              const float4 v = sg[q];
+              x[4 * q] = fmaf(y[4 * q], v.x, x[4 * q]);
+              x[4 * q + 1] = fmaf(y[4 * q + 1], v.y, x[4 * q + 1]);
+              x[4 * q + 2] = fmaf(y[4 * q + 2], v.z, x[4 * q + 2]);
+              x[4 * q + 3] = fmaf(y[4 * q + 3], v.w, x[4 * q + 3]);
+            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) x[q] = x[q] * f + y[q] * scale_log2;
+          }
         }
-        tmem_ld_16x32bx2_x32(s_taddr + 128, y);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) x[i] += y[i] * sck[i].z;
+        if (lane == 0 && q4 == 2 && i == 2) FP8_TRACE(7, t);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bars.sa_empty);
-      if (lane == 0 && q4 == 2) FP8_TRACE(7, t);
-      // pass B: group 3 and RoPE
-      if (!mbar_wait(bars.sb_full, t & 1, abort_flag)) { ok = false; return false; }
-      tc_fence_after();
-      if (lane == 0 && q4 == 2) FP8_TRACE(8, t);
-      if (work) {
-        float y[32], z[32];
-        tmem_ld_16x32bx2_x32(s_taddr + 0, y);
-        tmem_ld_16x32bx2_x32(s_taddr + 64, z);
-        const float f = rho * scale_log2;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) x[i] = (x[i] + y[i] * sck[i].w) * f + z[i] * scale_log2;
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bars.sb_empty);
       if (lane == 0 && q4 == 2) FP8_TRACE(9, t);
 
       float tmax = -INFINITY;
       if (work) {
-        const uint32_t vmask = static_cast<uint32_t>(info[s].mask[4 * half]) |
-                               (static_cast<uint32_t>(info[s].mask[4 * half + 1]) << 8) |
-                               (static_cast<uint32_t>(info[s].mask[4 * half + 2]) << 16) |
-                               (static_cast<uint32_t>(info[s].mask[4 * half + 3]) << 24);
         uint32_t m = vmask;
         if (causal && kPage * j + key0 + 31 >= lim) {
           const int nc = min(max(lim - kPage * j - key0, 0), 32);
           m &= nc >= 32 ? 0xFFFFFFFFu : ((1u << nc) - 1u);
         }
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          x[i] = ((m >> i) & 1u) ? x[i] : -INFINITY;
-          tmax = fmaxf(tmax, x[i]);
+        for (int i = 0; i < 32; ++i) x[i] = ((m >> i) & 1u) ? x[i] : -INFINITY;
+        // pairwise, so that the chain is five deep instead of 32
+        float mx[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) mx[i] = fmaxf(x[i], x[i + 16]);
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1) {
+#pragma unroll
+          for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
         }
+        tmax = mx[0];
       }
       tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
       const bool need = tmax > m_run + kRescaleThreshold;
@@ -736,13 +785,13 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
       // group exponents (the same in every thread, and in the gather warps
       // that scale V' with them)
       float4 beta;
-      const bool moved = gexp.update(info[s], beta);
+      const bool moved = gexp.update(gmax, beta);
       if (lane == 0 && q4 == 2) FP8_TRACE(13, t);
       if (__any_sync(0xffffffffu, any_pv && (alpha != 1.f || moved))) {
         // O holds every PV of the segment once PV(t-1), which frees its
         // stage, has completed (any_pv implies t > 0)
         const int tp = t - 1;
-        if (!mbar_wait(&bars.kv_empty[tp % kStages], (tp / kStages) & 1, abort_flag)) { ok = false; return false; }
+        if (!mbar_wait(&bars.kv_empty[tp % kStages], (tp / kStages) & 1, abort_flag, p.wait_ns)) { ok = false; return false; }
         tc_fence_after();
         if (warp_live) {
 #pragma unroll 1
@@ -760,21 +809,27 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
       if (lane == 0 && q4 == 2) FP8_TRACE(10, t);
       // P = exp2(s - m) as f16: this thread's 64-B half of row r of the
       // K-major swizzled P tile in the stage's RoPE chunk, whose last reader,
-      // pass B of this tile, has completed.  (P <= 2^8: the lazy max.)
+      // the RoPE part of this tile's QK^T, has completed.  (P <= 2^8: the
+      // lazy max.)
       const float m_safe = m_run == -INFINITY ? 0.f : m_run;
       uint8_t* stage = stage_ptr(smem, s);
       if (warp_live) {
         uint32_t pk[16];
         if (work) {
-          float lsum = 0.f;
+          float ps[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float a = fast_exp2(x[2 * i] - m_safe);
             const float b = fast_exp2(x[2 * i + 1] - m_safe);
-            lsum += a + b;
+            ps[i] = a + b;
             pk[i] = pack_f16x2(a, b);
           }
-          l_run += lsum;
+#pragma unroll
+          for (int w = 8; w >= 1; w >>= 1) {
+#pragma unroll
+            for (int i = 0; i < w; ++i) ps[i] += ps[i + w];
+          }
+          l_run += ps[0];
         } else {
 #pragma unroll
           for (int i = 0; i < 16; ++i) pk[i] = 0u;
@@ -797,7 +852,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
       if (j == je - 1) stage_next_q(u + 1);
       if (j == je - 1 && warp_live) {
         // ------------------------------------------------ epilogue of the segment
-        if (!mbar_wait(&bars.kv_empty[s], (t / kStages) & 1, abort_flag)) { ok = false; return false; }   // PV(t) done
+        if (!mbar_wait(&bars.kv_empty[s], (t / kStages) & 1, abort_flag, p.wait_ns)) { ok = false; return false; }   // PV(t) done
         tc_fence_after();
         const float l = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
         const bool has = any_pv && l > 0.f;
@@ -857,6 +912,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  FP8_SPAN(0);
 
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Smem::bar_off);
   Bars bars;
@@ -865,12 +921,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   bars.p_full = bar + 2 * kStages;
   bars.qk_done = bar + 3 * kStages;
   bars.v_ready = bar + 4 * kStages;
-  bars.sa_full = bar + 5 * kStages;
-  bars.sa_empty = bar + 5 * kStages + 1;
-  bars.sb_full = bar + 5 * kStages + 2;
-  bars.sb_empty = bar + 5 * kStages + 3;
-  bars.q_full = bar + 5 * kStages + 4;
-  bars.done = bar + 5 * kStages + 5;
+  bars.slot_full = bar + 5 * kStages;
+  bars.slot_empty = bar + 5 * kStages + kSlots;
+  bars.q_full = bar + 5 * kStages + 2 * kSlots;
+  bars.done = bar + 5 * kStages + 2 * kSlots + 1;
   StageInfo* info = reinterpret_cast<StageInfo*>(smem + Smem::info_off);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::misc_off + 4);
@@ -889,10 +943,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         info[s].gmax[w] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
-    mbar_init(bars.sa_full, 1);
-    mbar_init(bars.sa_empty, 4);
-    mbar_init(bars.sb_full, 1);
-    mbar_init(bars.sb_empty, 4);
+    for (int r = 0; r < kSlots; ++r) {
+      mbar_init(&bars.slot_full[r], 1);
+      mbar_init(&bars.slot_empty[r], 4);
+    }
     mbar_init(bars.q_full, 4);
     mbar_init(bars.done, 1);
     fence_barrier_init();
@@ -910,6 +964,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const Partition part = load_partition(p, blockIdx.x);
   if (threadIdx.x == 0) FP8_TRACE(15, 0);
+  FP8_SPAN(1);
 
   if (!*abort_flag) {
     if (warp == kWarpQPrefetch) {
@@ -925,6 +980,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) FP8_TRACE(15, 1);
+  FP8_SPAN(2);
   tc_fence_after();
   if (warp == kWarpMma) {
     __syncwarp();
@@ -938,6 +994,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 extern "C" __attribute__((visibility("default"))) int mla_trace_fp8_copy(void* host_dst, size_t bytes) {
   if (bytes > sizeof(g_fp8_trace)) bytes = sizeof(g_fp8_trace);
   return cudaMemcpyFromSymbol(host_dst, g_fp8_trace, bytes) == cudaSuccess ? 0 : 4;
+}
+extern "C" __attribute__((visibility("default"))) int mla_trace_fp8_span_copy(void* host_dst, size_t bytes) {
+  if (bytes > sizeof(g_fp8_span)) bytes = sizeof(g_fp8_span);
+  return cudaMemcpyFromSymbol(host_dst, g_fp8_span, bytes) == cudaSuccess ? 0 : 4;
 }
 #endif
 

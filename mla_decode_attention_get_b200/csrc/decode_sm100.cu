@@ -129,25 +129,52 @@ __device__ __forceinline__ int64_t q_tile_offset(const DecodeParams& p, const Un
   return q_tile_offset(p, ui, static_cast<int>(blockIdx.y) * kRows);
 }
 
+// One of a few values by a run-time index, without an indexed array (which
+// would live in local memory).
+__device__ __forceinline__ int pick(int i, int a, int b, int c, int d = 0) {
+  return i == 0 ? a : (i == 1 ? b : (i == 2 ? c : d));
+}
+
+// The last page the load warp issued into each stage (-1: none), so that a
+// CTA that gives up can wait for its own copies before it exits.
+struct Issued {
+  int t0 = -1, t1 = -1, t2 = -1;
+  __device__ __forceinline__ void set(int s, int t) {
+    if (s == 0) t0 = t;
+    else if (s == 1) t1 = t;
+    else t2 = t;
+  }
+  __device__ __forceinline__ int get(int s) const { return pick(s, t0, t1, t2); }
+};
+static_assert(kStages == 3, "Issued holds three stages");
+
 // ---------------------------------------------------------------------------
 // Warp 0 (one lane): TMA loads of cache pages with L2 warmed kPrefetchPages
 // ahead, and an L2 prefetch of the next segment's query tile.
 __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition& part, const CUtensorMap* tmap_kv,
-                                          uint8_t* smem, Bars bars, StageInfo* info, volatile int* abort_flag) {
+                                          uint8_t* smem, Bars bars, StageInfo* info, volatile int* abort_flag,
+                                          Issued& issued) {
   const uint64_t pol_kv = l2_policy_evict_first();
   const uint32_t q_bytes = static_cast<uint32_t>(tile_valid_rows(p)) * kDqk * 2;
   int t = 0;
-  int last_t[kStages];
-#pragma unroll
-  for (int s = 0; s < kStages; ++s) last_t[s] = -1;
   bool ok = true;
 
   // Physical pages of the next kPrefetchPages pages, read when they are
-  // warmed in L2 so that a page's TMA load never waits on the block table.
-  int ring[kPrefetchPages];
+  // warmed in L2 so that a page's TMA load never waits on the block table
+  // (four scalars: an indexed array would live in local memory).
+  static_assert(kPrefetchPages == 4, "the page ring holds four entries");
+  int r0 = -1, r1 = -1, r2 = -1, r3 = -1;
+  auto ring_set = [&](int j, int phys) {
+    const int i = j % kPrefetchPages;
+    if (i == 0) r0 = phys;
+    else if (i == 1) r1 = phys;
+    else if (i == 2) r2 = phys;
+    else r3 = phys;
+  };
+  auto ring_get = [&](int j) { return pick(j % kPrefetchPages, r0, r1, r2, r3); };
   auto fetch_ahead = [&](int b, int j) {
     const int phys = page_of(p, b, j);
-    ring[j % kPrefetchPages] = phys;
+    ring_set(j, phys);
     if (phys >= 0 && phys < p.num_blocks) {
 #pragma unroll 1
       for (int c = 0; c < kChunks; ++c) tma_prefetch_3d(tmap_kv, 64 * c, 0, phys);
@@ -165,9 +192,9 @@ __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition
       const UnitInfo ui = unit_info(p, u);
       // read the first pages' table entries together, then warm L2
       const int jn = min(je, jb + kPrefetchPages);
-      for (int j = jb; j < jn; ++j) ring[j % kPrefetchPages] = page_of(p, ui.b, j);
+      for (int j = jb; j < jn; ++j) ring_set(j, page_of(p, ui.b, j));
       for (int j = jb; j < jn; ++j) {
-        const int phys = ring[j % kPrefetchPages];
+        const int phys = ring_get(j);
         if (phys >= 0 && phys < p.num_blocks) {
 #pragma unroll 1
           for (int c = 0; c < kChunks; ++c) tma_prefetch_3d(tmap_kv, 64 * c, 0, phys);
@@ -175,10 +202,10 @@ __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition
       }
       for (int j = jb; j < je; ++j) {
         const int s = t % kStages;
-        if (!mbar_wait(&bars.kv_empty[s], ((t / kStages) & 1) ^ 1, abort_flag)) { ok = false; return false; }
+        if (!mbar_wait(&bars.kv_empty[s], ((t / kStages) & 1) ^ 1, abort_flag, p.wait_ns)) { ok = false; return false; }
         MLA_TRACE_EV(0, t);
         int nv = min(kPage, ui.L - kPage * j);
-        const int phys = ring[j % kPrefetchPages];
+        const int phys = ring_get(j);
         if (phys < 0 || phys >= p.num_blocks) {
           atomicOr(p.err, kErrBlockTable);
           nv = 0;
@@ -190,7 +217,7 @@ __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition
 #pragma unroll 1
           for (int c = 0; c < kChunks; ++c)
             tma_load_3d(dst + c * kChunkBytes, tmap_kv, &bars.kv_full[s], 64 * c, 0, phys, pol_kv);
-          last_t[s] = t;
+          issued.set(s, t);
         } else {
           mbar_arrive(&bars.kv_full[s]);
         }
@@ -201,17 +228,7 @@ __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition
     }
   });
 
-  if (!ok) {
-    raise_abort(abort_flag, p.err);
-    // Drain this warp's own copies before the CTA tears down.
-    const uint64_t t0 = globaltimer_ns();
-    for (int s = 0; s < kStages; ++s) {
-      if (last_t[s] < 0) continue;
-      while (!mbar_try_wait(&bars.kv_full[s], (last_t[s] / kStages) & 1) &&
-             globaltimer_ns() - t0 < kWaitTimeoutNs) {
-      }
-    }
-  }
+  if (!ok) raise_abort(abort_flag, p.err);
 }
 
 // ---------------------------------------------------------------------------
@@ -238,9 +255,9 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
   Cursor qk = cursor_begin(p, part);
   Cursor pv = qk;
   int o_seg = -1;
-  int qk_nv[kStages];
-#pragma unroll
-  for (int s = 0; s < kStages; ++s) qk_nv[s] = 0;
+  // valid keys of the page in each stage (scalars: an indexed array would
+  // live in local memory)
+  int nv0 = 0, nv1 = 0, nv2 = 0;
   bool ok = true;
   uint64_t t_idle = globaltimer_ns();
   uint32_t spins = 0;
@@ -257,7 +274,7 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
       if (lane == 0) MLA_TRACE_EV(3, pv.t);
       tc_fence_after();
       const int s = pv.t % kStages;
-      if (qk_nv[s] > 0) {
+      if (pick(s, nv0, nv1, nv2) > 0) {
         const bool acc0 = (o_seg == pv.seg);
         const uint64_t vd = v_desc0 + ((s * kPageBytes) >> 4);
         const uint64_t pd = p_desc0 + ((s * kPageBytes) >> 4);
@@ -287,7 +304,9 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
         if (lane == 0) MLA_TRACE_EV(2, qk.t);
         tc_fence_after();
         const int nv = info[s].nvalid;
-        qk_nv[s] = nv;
+        if (s == 0) nv0 = nv;
+        else if (s == 1) nv1 = nv;
+        else nv2 = nv;
         if (nv > 0) {
           const uint64_t kd = k_desc0 + ((s * kPageBytes) >> 4);
           const uint32_t d = tmem_s0 + sb * kPage;
@@ -311,7 +330,7 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
       spins = 0;
       t_idle = globaltimer_ns();
     } else if ((++spins & 255u) == 0) {
-      const bool give_up = *abort_flag || globaltimer_ns() - t_idle > kWaitTimeoutNs;
+      const bool give_up = *abort_flag || globaltimer_ns() - t_idle > p.wait_ns;
       if (__shfl_sync(0xffffffffu, give_up ? 1 : 0, 0)) {
         ok = false;
         break;
@@ -409,8 +428,8 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
     for (int j = jb; j < je; ++j) {
       const int s = t % kStages;
       const int sb = t & 1;
-      if (!mbar_wait(&bars.kv_full[s], (t / kStages) & 1, abort_flag)) { ok = false; return false; }
-      if (!mbar_wait(&bars.s_full[sb], (t >> 1) & 1, abort_flag)) { ok = false; return false; }
+      if (!mbar_wait(&bars.kv_full[s], (t / kStages) & 1, abort_flag, p.wait_ns)) { ok = false; return false; }
+      if (!mbar_wait(&bars.s_full[sb], (t >> 1) & 1, abort_flag, p.wait_ns)) { ok = false; return false; }
       if (lane == 0 && q4 == 2) MLA_TRACE_EV(4, t);
       tc_fence_after();
       const int nv = info[s].nvalid;
@@ -449,7 +468,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
           // O holds every PV of the segment once PV(t-1), which frees its
           // stage, has completed (any_pv implies t > 0)
           const int tp = t - 1;
-          if (!mbar_wait(&bars.kv_empty[tp % kStages], (tp / kStages) & 1, abort_flag)) { ok = false; return false; }
+          if (!mbar_wait(&bars.kv_empty[tp % kStages], (tp / kStages) & 1, abort_flag, p.wait_ns)) { ok = false; return false; }
           tc_fence_after();
           if (lane == 0 && q4 == 2) MLA_TRACE_EV(9, t);
 #pragma unroll 1
@@ -515,7 +534,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
       if (j == je - 1) stage_next_q(u + 1);
       if (j == je - 1 && warp_live) {
         // ------------------------------------------------ epilogue of the segment
-        if (!mbar_wait(&bars.kv_empty[s], (t / kStages) & 1, abort_flag)) { ok = false; return false; }   // PV(t) done
+        if (!mbar_wait(&bars.kv_empty[s], (t / kStages) & 1, abort_flag, p.wait_ns)) { ok = false; return false; }   // PV(t) done
         tc_fence_after();
         const float l = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
         const bool has = any_pv && l > 0.f;
@@ -622,9 +641,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) MLA_TRACE_EV(10, 0);
   if (threadIdx.x == 0) MLA_TRACE_SPAN(0);
 
+  Issued issued;
   if (!*abort_flag) {
     if (warp == kWarpLoad) {
-      if (lane == 0) load_role(p, part, &tmap_kv, smem, bars, info, abort_flag);
+      if (lane == 0) load_role(p, part, &tmap_kv, smem, bars, info, abort_flag, issued);
     } else if (warp == kWarpMma) {
       mma_role(p, part, smem, bars, info, tmem_base, abort_flag);
     } else {
@@ -632,6 +652,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   tc_fence_before();
+  __syncthreads();
+  // A CTA that gave up may still have page copies of its own in flight (the
+  // load lane may have issued every page before another role gave up): the
+  // load lane waits for them, bounded, before the shared memory is released.
+  if (warp == kWarpLoad && lane == 0 && *abort_flag) {
+    const uint64_t t0 = globaltimer_ns();
+    for (int s = 0; s < kStages; ++s) {
+      const int lt = issued.get(s);
+      if (lt < 0) continue;
+      while (!mbar_try_wait(&bars.kv_full[s], (lt / kStages) & 1) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      }
+    }
+  }
   __syncthreads();
   if (threadIdx.x == 0) MLA_TRACE_EV(10, 1);
   if (threadIdx.x == 0) MLA_TRACE_SPAN(1);

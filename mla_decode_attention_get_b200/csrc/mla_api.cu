@@ -10,6 +10,7 @@
 
 #include "mla_decode.h"
 #include "mla_kernels.cuh"
+#include "ptx_sm100.cuh"
 
 namespace {
 
@@ -95,6 +96,10 @@ bool encode_bf16_map(CUtensorMap* map, const void* base, uint64_t d1, uint64_t d
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Give-up limit of the kernels' pipeline waits for the calls that follow
+// (mla_set_pipeline_wait_limit); 0 = the default.
+std::atomic<uint64_t> g_wait_limit_ns{0};
+
 // Validates a decode call and fills the kernel parameters.
 int prepare(const mla_decode_args* a, Plan* pl, mla::DecodeParams* kp) {
   if (a == nullptr) return MLA_ERR_INVALID_ARG;
@@ -147,6 +152,8 @@ int prepare(const mla_decode_args* a, Plan* pl, mla::DecodeParams* kp) {
   kp->rows_per_unit = pl->rows_per_unit;
   kp->scale_log2 = a->softmax_scale * 1.4426950408889634f;
   kp->causal = a->causal ? 1 : 0;
+  const uint64_t lim = g_wait_limit_ns.load(std::memory_order_relaxed);
+  kp->wait_ns = lim ? lim : mla::kWaitTimeoutNs;
   return MLA_OK;
 }
 
@@ -241,6 +248,11 @@ int mla_fp8_cache_write(const void* k_new, int64_t k_row_stride, int32_t n, cons
                                                     static_cast<uint8_t*>(kv_cache), k_block_stride, num_blocks,
                                                     err_word, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_set_pipeline_wait_limit(uint64_t ns) {
+  g_wait_limit_ns.store(ns, std::memory_order_relaxed);
+  return MLA_OK;
 }
 
 const char* mla_status_string(int status) {

@@ -51,6 +51,7 @@ struct DecodeParams {
   int rows_per_unit;
   float scale_log2;           // softmax_scale * log2(e)
   int causal;
+  uint64_t wait_ns;           // give-up limit of the pipeline waits (drains keep kWaitTimeoutNs)
 };
 
 // Launch with programmatic stream serialization: the kernel may start while

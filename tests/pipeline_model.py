@@ -29,8 +29,9 @@ catch it:
   committed per page, with parity t & 1.
 
 `Fp8Model` (at the end) does the same for the FP8 kernel in
-`csrc/decode_fp8_sm100.cu`, whose protocol differs (two stages filled by 8
-gather warps, QK^T in two passes, P' tiles in the stage).
+`csrc/decode_fp8_sm100.cu`, whose protocol differs (three stages filled by 8
+gather warps, QK^T in five parts through a ring of three TMEM slots, V'
+rewritten in place by the gather warps).
 """
 from __future__ import annotations
 
@@ -41,6 +42,8 @@ from typing import Dict, List, Optional
 STAGES = 3
 WARPS = 4            # softmax warps, one per TMEM lane quadrant
 GATHER_WARPS = 8     # FP8 kernel
+FP8_PARTS = 5        # FP8 kernel: QK^T parts per tile (latent groups 0-3, RoPE)
+FP8_SLOTS = 3        # FP8 kernel: partial-S slots in TMEM
 
 
 class ProtocolError(AssertionError):
@@ -328,9 +331,12 @@ FP8_STAGES = 3
 
 class Fp8Model:
     """Random interleavings of the FP8 kernel's roles; the same checks as
-    `Model`.  `mutation`:
-    - "no_sa_wait": pass B does not wait for the softmax to read pass A;
-    - "early_p": the softmax writes P before pass B has completed;
+    `Model`.  Part i of tile t is QK^T item n = 5 t + i, written into slot
+    n % 3 (use n // 3 of the slot).  `mutation`:
+    - "no_slot_wait": the MMA writes a slot without waiting for the softmax
+      to have read its previous part;
+    - "early_p": the softmax writes P before the RoPE part of QK^T (the last
+      reader of the chunk P goes to) has completed;
     - "early_v": the gather rewrites V' without waiting for qk_done;
     - "no_seg_end_pv": PV of a segment's last tile waits for the next tile."""
 
@@ -350,18 +356,18 @@ class Fp8Model:
         self.p_full = [Barrier(f"p_full[{s}]", WARPS) for s in range(S)]
         self.qk_done = [Barrier(f"qk_done[{s}]", 1) for s in range(S)]
         self.v_ready = [Barrier(f"v_ready[{s}]", GATHER_WARPS) for s in range(S)]
-        self.sa_full, self.sa_empty = Barrier("sa_full", 1), Barrier("sa_empty", WARPS)
-        self.sb_full, self.sb_empty = Barrier("sb_full", 1), Barrier("sb_empty", WARPS)
+        self.slot_full = [Barrier(f"slot_full[{r}]", 1) for r in range(FP8_SLOTS)]
+        self.slot_empty = [Barrier(f"slot_empty[{r}]", WARPS) for r in range(FP8_SLOTS)]
         self.q_full = Barrier("q_full", WARPS)
         self.pipe: List[tuple] = []
         self.stage_page: List[Optional[int]] = [None] * S
         self.stage_writers = [0] * S
         self.v_writers = [0] * S
         self.codes_are_v = [False] * S        # the stage's codes were rewritten as V'
-        self.rope_is_p = [False] * S          # the RoPE chunk holds P (pass B of its tile is over)
-        self.buf = [None, None, None]         # (tile, pass) held by each partial-S buffer
-        self.reading = [set(), set(), set()]
-        self.qka_done, self.qkb_done, self.pv_done = set(), set(), set()
+        self.rope_is_p = [False] * S          # the RoPE chunk holds P (QK^T of its tile is over)
+        self.slot = [None] * FP8_SLOTS        # (tile, part) held by each slot
+        self.reading = [set() for _ in range(FP8_SLOTS)]
+        self.qk_all_done, self.pv_done = set(), set()
         self.p_written: Dict[int, int] = {}
         self.q_writes: Dict[int, int] = {}
         self.q_seg = -1
@@ -400,7 +406,7 @@ class Fp8Model:
             yield ("wait", lambda s=s, t=t: self.qk_done[s].passes(t // FP8_STAGES))
         if self.stage_page[s] != t:
             raise ProtocolError(f"V' of tile {t} rewrites stage {s} holding {self.stage_page[s]}")
-        if t not in self.qkb_done:
+        if t not in self.qk_all_done:
             raise ProtocolError(f"V' of tile {t} rewrites codes that QK^T still reads")
         yield ("step",)
         self.v_writers[s] += 1
@@ -417,13 +423,13 @@ class Fp8Model:
             yield ("wait", lambda s=s, t=t: self.kv_full[s].passes(ph(t)))
             if t in self.first_of_seg:
                 yield ("wait", lambda t=t: self.q_full.passes(self.seg_of[t]))
-            yield ("wait", lambda t=t: self.sb_empty.passes(t - 1))
-            self.pipe.append(("QKA", t))
-            self.pipe.append(("commit", self.sa_full, t))
-            if self.mut != "no_sa_wait":
-                yield ("wait", lambda t=t: self.sa_empty.passes(t))
-            self.pipe.append(("QKB", t))
-            self.pipe.append(("commit", self.sb_full, t))
+            for i in range(FP8_PARTS):
+                n = FP8_PARTS * t + i
+                r, use = n % FP8_SLOTS, n // FP8_SLOTS
+                if self.mut != "no_slot_wait":
+                    yield ("wait", lambda r=r, use=use: self.slot_empty[r].passes(use - 1))
+                self.pipe.append(("QK", t, i, r))
+                self.pipe.append(("commit", self.slot_full[r], use))
             self.pipe.append(("commit", self.qk_done[s], ph(t)))
             if prev is not None:
                 yield from self._pv(prev)
@@ -442,6 +448,13 @@ class Fp8Model:
         self.pipe.append(("PV", t))
         self.pipe.append(("commit", self.kv_empty[s], t // FP8_STAGES))
 
+    def _write_p(self, w, t, s):
+        if t not in self.qk_all_done or self.stage_page[s] != t:
+            raise ProtocolError(f"softmax {w} writes P of tile {t} into a RoPE chunk QK^T still reads")
+        yield ("step",)
+        self.rope_is_p[s] = True
+        self.p_written[t] = self.p_written.get(t, 0) + 1
+
     def softmax(self, w):
         live = w < self.plan.live_warps
         self._stage_q(0)
@@ -453,29 +466,22 @@ class Fp8Model:
             for j in range(n):
                 s = t % FP8_STAGES
                 yield ("wait", lambda s=s, t=t: self.kv_full[s].passes(t // FP8_STAGES))
-                yield ("wait", lambda t=t: self.sa_full.passes(t))
-                if live:
-                    for b in range(3):
-                        if self.buf[b] != (t, "A"):
-                            raise ProtocolError(f"softmax {w} reads buffer {b} for pass A of tile {t}, "
-                                                f"holding {self.buf[b]}")
-                        self.reading[b].add(w)
-                    yield ("step",)
-                    for b in range(3):
-                        self.reading[b].discard(w)
-                self.sa_empty.arrive(t)
-                if self.mut != "early_p":
-                    yield ("wait", lambda t=t: self.sb_full.passes(t))
+                wrote_p = False
+                for i in range(FP8_PARTS):
+                    if i == FP8_PARTS - 1 and self.mut == "early_p" and live:
+                        yield from self._write_p(w, t, s)
+                        wrote_p = True
+                    q = FP8_PARTS * t + i
+                    r, use = q % FP8_SLOTS, q // FP8_SLOTS
+                    yield ("wait", lambda r=r, use=use: self.slot_full[r].passes(use))
                     if live:
-                        for b in range(2):
-                            if self.buf[b] != (t, "B"):
-                                raise ProtocolError(f"softmax {w} reads buffer {b} for pass B of tile {t}, "
-                                                    f"holding {self.buf[b]}")
-                            self.reading[b].add(w)
+                        if self.slot[r] != (t, i):
+                            raise ProtocolError(f"softmax {w} reads slot {r} for part {i} of tile {t}, "
+                                                f"holding {self.slot[r]}")
+                        self.reading[r].add(w)
                         yield ("step",)
-                        for b in range(2):
-                            self.reading[b].discard(w)
-                    self.sb_empty.arrive(t)
+                        self.reading[r].discard(w)
+                    self.slot_empty[r].arrive(use)
                 need = live and any_pv and bool((self.plan.rescale or {}).get((w, t), False))
                 if need:
                     yield ("wait", lambda t=t: self.kv_empty[(t - 1) % FP8_STAGES].passes((t - 1) // FP8_STAGES))
@@ -484,20 +490,13 @@ class Fp8Model:
                     self.o_busy.add(w)
                     yield ("step",)
                     self.o_busy.discard(w)
-                if live:
-                    if t not in self.qkb_done or self.stage_page[s] != t:
-                        raise ProtocolError(f"softmax {w} writes P of tile {t} into a RoPE chunk pass B still reads")
-                    yield ("step",)
-                    self.rope_is_p[s] = True
-                    self.p_written[t] = self.p_written.get(t, 0) + 1
-                if self.mut == "early_p":
-                    yield ("wait", lambda t=t: self.sb_full.passes(t))
-                    self.sb_empty.arrive(t)
+                if live and not wrote_p:
+                    yield from self._write_p(w, t, s)
                 self.p_full[s].arrive(t // FP8_STAGES)
                 any_pv = True
                 if j == n - 1:
                     if k + 1 < len(self.plan.segments):
-                        if t not in self.qkb_done:
+                        if t not in self.qk_all_done:
                             raise ProtocolError(f"softmax {w} overwrites the query tile while QK of tile {t} runs")
                         self._stage_q(k + 1)
                         yield ("step",)
@@ -527,20 +526,19 @@ class Fp8Model:
         s = t % FP8_STAGES
         if self.stage_page[s] != t:
             raise ProtocolError(f"{kind} of tile {t} reads stage {s} holding {self.stage_page[s]}")
-        if kind in ("QKA", "QKB"):
+        if kind == "QK":
+            i, r = item[2], item[3]
             if self.q_seg != self.seg_of[t]:
-                raise ProtocolError(f"{kind} of tile {t} reads the query tile of segment {self.q_seg}")
+                raise ProtocolError(f"QK part {i} of tile {t} reads the query tile of segment {self.q_seg}")
             if self.codes_are_v[s]:
-                raise ProtocolError(f"{kind} of tile {t} reads codes already rewritten as V'")
-            bufs = (0, 1, 2) if kind == "QKA" else (0, 1)
-            for b in bufs:
-                if self.reading[b]:
-                    raise ProtocolError(f"{kind} of tile {t} overwrites buffer {b} while it is being read")
-            if kind == "QKB" and self.rope_is_p[s]:
-                raise ProtocolError(f"QKB of tile {t} reads a RoPE chunk that holds P")
-            for b in bufs:
-                self.buf[b] = (t, "A" if kind == "QKA" else "B")
-            (self.qka_done if kind == "QKA" else self.qkb_done).add(t)
+                raise ProtocolError(f"QK part {i} of tile {t} reads codes already rewritten as V'")
+            if self.reading[r]:
+                raise ProtocolError(f"QK part {i} of tile {t} overwrites slot {r} while it is being read")
+            if i == FP8_PARTS - 1 and self.rope_is_p[s]:
+                raise ProtocolError(f"QK RoPE part of tile {t} reads a RoPE chunk that holds P")
+            self.slot[r] = (t, i)
+            if i == FP8_PARTS - 1:
+                self.qk_all_done.add(t)
         else:
             if self.p_written.get(t, 0) != self.plan.live_warps:
                 raise ProtocolError(f"PV of tile {t} reads P before every live warp wrote it")

@@ -44,11 +44,13 @@ def test_boosted_rows_with_their_own_scales(case):
 
 def _writer_cache(w, rng, lo, hi):
     """Replace w's FP8 cache by rows quantised with the writer's rule from bf16
-    rows whose per-group max |x| is log-uniform in [lo, hi]."""
+    rows whose per-group max |x| is log-uniform in [lo, hi]; the 64 RoPE dims
+    of a row get a max |x| from the same range (they enter the logits
+    unscaled, so their magnitude has to follow the latent part's)."""
     n = w.kv_fp8.shape[0] * 64
     x = rng.standard_normal((n, 576)).astype(np.float32)
-    for g in range(4):
-        grp = x[:, 128 * g:128 * (g + 1)]
+    for lo_d, hi_d in [(0, 128), (128, 256), (256, 384), (384, 512), (512, 576)]:
+        grp = x[:, lo_d:hi_d]
         target = np.exp(rng.uniform(np.log(lo), np.log(hi), size=(n, 1))).astype(np.float32)
         grp *= target / np.abs(grp).max(axis=1, keepdims=True)
     k_bits = I.f32_to_bf16_bits(x)
@@ -73,7 +75,10 @@ def test_writer_made_small_scales(case, q_gain):
     w.q_bits = I.f32_to_bf16_bits(q)
     out, lse, err = run(w)
     assert err == 0
-    assert_close(out, lse, *oracle(w))
+    ref_out, ref_lse = oracle(w)
+    # moderate logits: the absolute lse bar is then far above fp32's own ulp
+    assert np.abs(ref_lse[np.isfinite(ref_lse)]).max() < 64.0
+    assert_close(out, lse, ref_out, ref_lse)
 
 
 @pytest.mark.parametrize("case", ["dense", "sparse"])

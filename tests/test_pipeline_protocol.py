@@ -1,8 +1,8 @@
 """The decode kernels' barrier protocols, checked on host-side models (CPU).
 
 `pipeline_model` restates the hand-offs of one CTA of the bf16 decode kernel
-(and, in `Fp8Model`, of the FP8 kernel, with its two-pass QK^T and the V'
-rewrite by the gather warps):
+(and, in `Fp8Model`, of the FP8 kernel, with its five-part QK^T through a
+ring of three TMEM slots and the V' rewrite by the gather warps):
 - the page producer: TMA, or 8 gather warps on the FP8 kernel;
 - the MMA warp's event loop;
 - four softmax warps, with padding warps, lazy rescales, segment epilogues and
@@ -48,7 +48,7 @@ def test_fp8_protocol_runs_clean_on_random_schedules():
         PM.Fp8Model(PM.Plan([1, 1, 1, 1, 1], 4, True, {}), seed).run()
 
 
-@pytest.mark.parametrize("mutation", ["no_sa_wait", "early_p", "early_v", "no_seg_end_pv"])
+@pytest.mark.parametrize("mutation", ["no_slot_wait", "early_p", "early_v", "no_seg_end_pv"])
 def test_fp8_planted_mistakes_are_caught(mutation):
     caught = 0
     for seed in range(60):
