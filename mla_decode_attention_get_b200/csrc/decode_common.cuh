@@ -11,7 +11,7 @@ namespace dec {
 
 constexpr int kPageBytes = kPage * kDqk * 2;  // 73728: 64 tokens x 576 bf16
 constexpr int kChunkBytes = kPage * 128;      // 8192: 64 rows x 64 dims (one 128-B swizzle column)
-constexpr int kPrefetchPages = 4;             // pages warmed in L2 ahead of the TMA loads
+constexpr int kPrefetchPages = 4;             // block-table entries read ahead of the TMA loads
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr int kErrBlockTable = 1, kErrIndex = 2, kErrTimeout = 4, kErrSeqlen = 8, kErrInternal = 16;

@@ -48,7 +48,6 @@
 //    drains its own MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
-#include <cuda_fp8.h>
 
 #include "decode_common.cuh"
 #include "mla_kernels.cuh"
@@ -59,7 +58,7 @@ namespace mla {
 #ifdef MLA_TRACE
 // Opt-in pipeline trace (built only with -DMLA_TRACE): clock64() stamps of the
 // hand-offs of every tile in the first kFp8TraceCtas CTAs of row tile 0.
-constexpr int kFp8TraceCtas = 4, kFp8TraceEvents = 16, kFp8TraceTiles = 256;
+constexpr int kFp8TraceCtas = 4, kFp8TraceEvents = 64, kFp8TraceTiles = 256;
 __device__ unsigned long long g_fp8_trace[kFp8TraceCtas][kFp8TraceEvents][kFp8TraceTiles];
 // Per CTA (all of them): %globaltimer at entry, after the set-up and the
 // dependency wait, and at exit, and the SM it ran on.
@@ -113,6 +112,16 @@ constexpr int kRescaleGroupLog2 = 7;           // raise E_g once a scale reaches
 
 constexpr int kWarpQPrefetch = 0, kWarpMma = 1, kWarpSoftmax0 = 2, kWarpGather0 = 6;
 constexpr int kGatherWarps = 8;                // warp gw converts keys [8 gw, 8 gw + 8)
+// The V' rewrite is left to the four gather warps whose schedulers hold
+// neither the MMA warp nor the prefetch warp (gather warps 0, 1, 4, 5 on
+// schedulers 2 and 3), 16 keys each: the softmax warp that shares a scheduler
+// with the MMA warp is the slowest one, and a quarter of a gather warp's
+// instructions are the rewrite.
+constexpr int kRewriteWarps = 4;
+__host__ __device__ constexpr int rewrite_index(int gw) { return (gw & 2) ? -1 : ((gw >> 2) << 1) | (gw & 1); }
+static_assert(rewrite_index(0) == 0 && rewrite_index(1) == 1 && rewrite_index(4) == 2 && rewrite_index(5) == 3 &&
+                  rewrite_index(2) < 0 && rewrite_index(3) < 0 && rewrite_index(6) < 0 && rewrite_index(7) < 0,
+              "four rewriting warps, one per 16 keys");
 constexpr int kThreads = 32 * (kWarpGather0 + kGatherWarps);
 
 struct StageInfo {
@@ -140,7 +149,7 @@ struct Bars {
   uint64_t* kv_empty;   // [stage] PV of the stage's tile completed (commit)
   uint64_t* p_full;     // [stage] P of the stage's tile written (4 softmax warps)
   uint64_t* qk_done;    // [stage] both QK^T passes of the stage's tile completed (commit)
-  uint64_t* v_ready;    // [stage] V' of the stage's tile written (8 gather warps)
+  uint64_t* v_ready;    // [stage] V' of the stage's tile written (4 rewriting gather warps)
   uint64_t* slot_full;  // [slot] a part of QK^T completed into the slot (commit)
   uint64_t* slot_empty; // [slot] the slot was read (4 softmax warps)
   uint64_t* q_full;     // query tile of the next segment in TMEM (4 softmax warps)
@@ -260,9 +269,10 @@ __device__ __forceinline__ void q_prefetch_role(const DecodeParams& p, const Par
 // table entries of tile t+2 and the indices of tile t+3 are in flight.  Lane
 // l converts codes [8 l, 8 l + 8) and [256 + 8 l, 256 + 8 l + 8) and, for
 // l < 16, copies RoPE dims [512 + 4 l, +4) of each of the warp's 8 rows.
-// After converting tile t the warps rewrite tile t-1 as V' (they wait for its
-// QK^T to complete): lane l scales key 8 gw + l / 4, group l % 4 (128 codes,
-// 16 x 16 B) by its scale x 2^-E_g.  So PV of tile t-1 can run while tile t+1
+// After converting tile t the rewriting warps rewrite tile t-1 as V' (they
+// wait for its QK^T to complete): lane l of rewriter rw scales key
+// 16 rw + 8 h + l / 4, group l % 4 (128 codes, 16 x 16 B), h = 0, 1, by its
+// scale x 2^-E_g.  So PV of tile t-1 can run while tile t+1
 // converts, and the stage it frees is the one tile t+2 needs.
 __device__ __forceinline__ void gather_role(const DecodeParams& p, const Partition& part, uint8_t* smem, Bars bars,
                                             volatile int* abort_flag, int gw) {
@@ -312,6 +322,7 @@ __device__ __forceinline__ void gather_role(const DecodeParams& p, const Partiti
   };
 
   // V' of tile tr (cursor rwc), one tile behind the conversion
+  const int rw = rewrite_index(gw);
   Cursor rwc = cursor_begin(p, part);
   int tr = 0, rw_seg = -1;
   GroupExp gexp;
@@ -326,22 +337,25 @@ __device__ __forceinline__ void gather_role(const DecodeParams& p, const Partiti
     float4 beta;
     gexp.update(GroupExp::tile_max(info[s]), beta);
     const int e = lane >> 2, qq = lane & 3;
-    const int k = 8 * gw + e;
-    const float sk = scales[scale_index(s, qq, k)];
-    const float f32 = sk * pow2i(-gexp.e(qq));
-    const uint32_t f = pack_f16x2(f32, f32);
-    uint8_t* row = stage_ptr(smem, s) + k * 128;
+    const float gsc = pow2i(-gexp.e(qq));
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h) {
+      const int k = 16 * rw + 8 * h + e;
+      const float f32 = scales[scale_index(s, qq, k)] * gsc;
+      const uint32_t f = pack_f16x2(f32, f32);
+      uint8_t* row = stage_ptr(smem, s) + k * 128;
 #pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      uint4* base = reinterpret_cast<uint4*>(row + (2 * qq + cc) * kChunkBytes);
-      // a quarter warp (two keys x four groups) touches eight different 16-B banks
-      uint4 v[8];
+      for (int cc = 0; cc < 2; ++cc) {
+        uint4* base = reinterpret_cast<uint4*>(row + (2 * qq + cc) * kChunkBytes);
+        // a quarter warp (two keys x four groups) touches eight different 16-B banks
+        uint4 v[8];
 #pragma unroll
-      for (int uu = 0; uu < 8; ++uu) v[uu] = base[(uu + 2 * qq + e) & 7];
+        for (int uu = 0; uu < 8; ++uu) v[uu] = base[(uu + 2 * qq + e) & 7];
 #pragma unroll
-      for (int uu = 0; uu < 8; ++uu)
-        base[(uu + 2 * qq + e) & 7] =
-            make_uint4(hmul2_f16(v[uu].x, f), hmul2_f16(v[uu].y, f), hmul2_f16(v[uu].z, f), hmul2_f16(v[uu].w, f));
+        for (int uu = 0; uu < 8; ++uu)
+          base[(uu + 2 * qq + e) & 7] =
+              make_uint4(hmul2_f16(v[uu].x, f), hmul2_f16(v[uu].y, f), hmul2_f16(v[uu].z, f), hmul2_f16(v[uu].w, f));
+      }
     }
     fence_proxy_async_smem();
     __syncwarp();
@@ -415,13 +429,8 @@ __device__ __forceinline__ void gather_role(const DecodeParams& p, const Partiti
           const uint2 codes = half ? n1[e] : n0[e];
           const uint32_t w[2] = {codes.x, codes.y};
           uint32_t o[4];
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] & 0xFFFFu), __NV_E4M3);
-            const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] >> 16), __NV_E4M3);
-            o[2 * i] = *reinterpret_cast<const uint32_t*>(&lo);
-            o[2 * i + 1] = *reinterpret_cast<const uint32_t*>(&hi);
-          }
+          e4m3x4_to_f16x4(w[0], o[0], o[1]);
+          e4m3x4_to_f16x4(w[1], o[2], o[3]);
           const int chunk = 4 * half + (lane >> 3);
           st_shared_v4(rowa + chunk * kChunkBytes + slot, make_uint4(o[0], o[1], o[2], o[3]));
         }
@@ -461,9 +470,9 @@ __device__ __forceinline__ void gather_role(const DecodeParams& p, const Partiti
     pend_n = pend_nn;
     pos_nn = pos_nnn;
     ++t;
-    if (t - tr > 1 && !rewrite()) { ok = false; break; }
+    if (rw >= 0 && t - tr > 1 && !rewrite()) { ok = false; break; }
   }
-  while (ok && rwc.valid) {
+  while (ok && rw >= 0 && rwc.valid) {
     if (!rewrite()) ok = false;
   }
   if (!ok && lane == 0) raise_abort(abort_flag, p.err);
@@ -511,7 +520,9 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
   int o_seg = -1;
   auto pv_tile = [&](int t, int seg, int nv) -> bool {
     const int s = t % kStages;
+    FP8_TRACE(41, t);
     if (!mbar_wait(&bars.p_full[s], (t / kStages) & 1, abort_flag, p.wait_ns)) return false;
+    FP8_TRACE(42, t);
     if (!mbar_wait(&bars.v_ready[s], (t / kStages) & 1, abort_flag, p.wait_ns)) return false;
     tc_fence_after();
     FP8_TRACE(5, t);
@@ -551,6 +562,7 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
     const uint64_t kd = k_desc0 + ((s * kStageBytes) >> 4);
 #pragma unroll 1
     for (int i = 0; i < kParts; ++i) {
+      FP8_TRACE(16 + 5 * i, t);
       if (!mbar_wait(&bars.slot_empty[ring.slot], ring.phase ^ 1u, abort_flag, p.wait_ns)) {
         ok = false;
         break;
@@ -568,6 +580,7 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
         }
       }
       umma_commit_elect(&bars.slot_full[ring.slot]);
+      FP8_TRACE(17 + 5 * i, t);
       ring.next();
     }
     if (!ok) break;
@@ -722,8 +735,11 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
       for (int i = 0; i < 32; ++i) x[i] = 0.f;
 #pragma unroll 1
       for (int i = 0; i < kParts; ++i) {
+        if (lane == 0 && q4 == 2) FP8_TRACE(18 + 5 * i, t);
+        if (lane == 0 && i == 0) FP8_TRACE(47 + q4, t);
         if (!mbar_wait(&bars.slot_full[ring.slot], ring.phase, abort_flag, p.wait_ns)) { ok = false; return false; }
         tc_fence_after();
+        if (lane == 0 && q4 == 2) FP8_TRACE(19 + 5 * i, t);
         if (lane == 0 && q4 == 2 && i == 0) FP8_TRACE(6, t);
         if (lane == 0 && q4 == 2 && i == kParts - 1) FP8_TRACE(8, t);
         float y[32];
@@ -731,6 +747,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.slot_empty[ring.slot]);
+        if (lane == 0 && i == 0) FP8_TRACE(43 + q4, t);
         ring.next();
         if (work) {
           if (i < 4) {
@@ -749,6 +766,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
           }
         }
         if (lane == 0 && q4 == 2 && i == 2) FP8_TRACE(7, t);
+        if (lane == 0 && q4 == 2) FP8_TRACE(20 + 5 * i, t);
       }
       if (lane == 0 && q4 == 2) FP8_TRACE(9, t);
 
@@ -846,6 +864,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.p_full[s]);
+      if (lane == 0) FP8_TRACE(51 + q4, t);
       if (lane == 0 && q4 == 2) FP8_TRACE(11, t);
       if (nv > 0) any_pv = true;
 
@@ -937,7 +956,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.kv_empty[s], 1);
       mbar_init(&bars.p_full[s], 4);
       mbar_init(&bars.qk_done[s], 1);
-      mbar_init(&bars.v_ready[s], kGatherWarps);
+      mbar_init(&bars.v_ready[s], kRewriteWarps);
       for (int w = 0; w < kGatherWarps; ++w) {
         info[s].mask[w] = 0;
         info[s].gmax[w] = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -149,8 +149,10 @@ struct Issued {
 static_assert(kStages == 3, "Issued holds three stages");
 
 // ---------------------------------------------------------------------------
-// Warp 0 (one lane): TMA loads of cache pages with L2 warmed kPrefetchPages
-// ahead, and an L2 prefetch of the next segment's query tile.
+// Warp 0 (one lane): TMA loads of cache pages, their block-table entries
+// read kPrefetchPages pages ahead, and an L2 prefetch of the next segment's
+// query tile.  (Warming the pages themselves in L2 ahead of their loads, 1 to
+// 4 pages ahead, measured slower than not warming them at all.)
 __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition& part, const CUtensorMap* tmap_kv,
                                           uint8_t* smem, Bars bars, StageInfo* info, volatile int* abort_flag,
                                           Issued& issued) {
@@ -172,14 +174,6 @@ __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition
     else r3 = phys;
   };
   auto ring_get = [&](int j) { return pick(j % kPrefetchPages, r0, r1, r2, r3); };
-  auto fetch_ahead = [&](int b, int j) {
-    const int phys = page_of(p, b, j);
-    ring_set(j, phys);
-    if (phys >= 0 && phys < p.num_blocks) {
-#pragma unroll 1
-      for (int c = 0; c < kChunks; ++c) tma_prefetch_3d(tmap_kv, 64 * c, 0, phys);
-    }
-  };
 
   for_each_segment(p, part, [&](int u, int jb, int je) -> bool {
     // warm the query tile of the following segment
@@ -190,16 +184,9 @@ __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition
     }
     {
       const UnitInfo ui = unit_info(p, u);
-      // read the first pages' table entries together, then warm L2
+      // read the first pages' table entries together
       const int jn = min(je, jb + kPrefetchPages);
       for (int j = jb; j < jn; ++j) ring_set(j, page_of(p, ui.b, j));
-      for (int j = jb; j < jn; ++j) {
-        const int phys = ring_get(j);
-        if (phys >= 0 && phys < p.num_blocks) {
-#pragma unroll 1
-          for (int c = 0; c < kChunks; ++c) tma_prefetch_3d(tmap_kv, 64 * c, 0, phys);
-        }
-      }
       for (int j = jb; j < je; ++j) {
         const int s = t % kStages;
         if (!mbar_wait(&bars.kv_empty[s], ((t / kStages) & 1) ^ 1, abort_flag, p.wait_ns)) { ok = false; return false; }
@@ -221,7 +208,7 @@ __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition
         } else {
           mbar_arrive(&bars.kv_full[s]);
         }
-        if (j + kPrefetchPages < je) fetch_ahead(ui.b, j + kPrefetchPages);
+        if (j + kPrefetchPages < je) ring_set(j + kPrefetchPages, page_of(p, ui.b, j + kPrefetchPages));
         ++t;
       }
       return true;

@@ -44,6 +44,7 @@ WARPS = 4            # softmax warps, one per TMEM lane quadrant
 GATHER_WARPS = 8     # FP8 kernel
 FP8_PARTS = 5        # FP8 kernel: QK^T parts per tile (latent groups 0-3, RoPE)
 FP8_SLOTS = 3        # FP8 kernel: partial-S slots in TMEM
+FP8_REWRITERS = (0, 1, 4, 5)   # FP8 kernel: the gather warps that rewrite V'
 
 
 class ProtocolError(AssertionError):
@@ -355,7 +356,7 @@ class Fp8Model:
         self.kv_empty = [Barrier(f"kv_empty[{s}]", 1) for s in range(S)]
         self.p_full = [Barrier(f"p_full[{s}]", WARPS) for s in range(S)]
         self.qk_done = [Barrier(f"qk_done[{s}]", 1) for s in range(S)]
-        self.v_ready = [Barrier(f"v_ready[{s}]", GATHER_WARPS) for s in range(S)]
+        self.v_ready = [Barrier(f"v_ready[{s}]", len(FP8_REWRITERS)) for s in range(S)]
         self.slot_full = [Barrier(f"slot_full[{r}]", 1) for r in range(FP8_SLOTS)]
         self.slot_empty = [Barrier(f"slot_empty[{r}]", WARPS) for r in range(FP8_SLOTS)]
         self.q_full = Barrier("q_full", WARPS)
@@ -393,10 +394,10 @@ class Fp8Model:
                 self.codes_are_v[s] = False
             self.kv_full[s].arrive(ph(t))
             yield ("step",)
-            while t + 1 - tr > 1:
+            while w in FP8_REWRITERS and t + 1 - tr > 1:
                 yield from self._rewrite(tr)
                 tr += 1
-        while tr < self.T:
+        while w in FP8_REWRITERS and tr < self.T:
             yield from self._rewrite(tr)
             tr += 1
 
@@ -410,7 +411,7 @@ class Fp8Model:
             raise ProtocolError(f"V' of tile {t} rewrites codes that QK^T still reads")
         yield ("step",)
         self.v_writers[s] += 1
-        if self.v_writers[s] == GATHER_WARPS:
+        if self.v_writers[s] == len(FP8_REWRITERS):
             self.v_writers[s] = 0
             self.codes_are_v[s] = True
         self.v_ready[s].arrive(t // FP8_STAGES)
