@@ -112,16 +112,25 @@ constexpr int kRescaleGroupLog2 = 7;           // raise E_g once a scale reaches
 
 constexpr int kWarpQPrefetch = 0, kWarpMma = 1, kWarpSoftmax0 = 2, kWarpGather0 = 6;
 constexpr int kGatherWarps = 8;                // warp gw converts keys [8 gw, 8 gw + 8)
-// The V' rewrite is left to the four gather warps whose schedulers hold
-// neither the MMA warp nor the prefetch warp (gather warps 0, 1, 4, 5 on
-// schedulers 2 and 3), 16 keys each: the softmax warp that shares a scheduler
-// with the MMA warp is the slowest one, and a quarter of a gather warp's
-// instructions are the rewrite.
-constexpr int kRewriteWarps = 4;
-__host__ __device__ constexpr int rewrite_index(int gw) { return (gw & 2) ? -1 : ((gw >> 2) << 1) | (gw & 1); }
-static_assert(rewrite_index(0) == 0 && rewrite_index(1) == 1 && rewrite_index(4) == 2 && rewrite_index(5) == 3 &&
-                  rewrite_index(2) < 0 && rewrite_index(3) < 0 && rewrite_index(6) < 0 && rewrite_index(7) < 0,
-              "four rewriting warps, one per 16 keys");
+// The V' rewrite is left to the gather warps whose schedulers do not hold the
+// MMA warp (the softmax warp that shares a scheduler with the MMA warp is the
+// slowest one, and a quarter of a gather warp's instructions are the
+// rewrite): gather warps 2 and 6 (scheduler 0, whose prefetch warp is idle)
+// take 8 keys each, gather warps 0, 4 (scheduler 2) and 1, 5 (scheduler 3) 12.
+constexpr int kRewriteWarps = 6;
+struct RewriteKeys {
+  int first, count;
+};
+__host__ __device__ constexpr RewriteKeys rewrite_keys(int gw) {
+  return gw == 2 ? RewriteKeys{0, 8} : gw == 6 ? RewriteKeys{8, 8} : gw == 0 ? RewriteKeys{16, 12}
+         : gw == 4 ? RewriteKeys{28, 12} : gw == 1 ? RewriteKeys{40, 12} : gw == 5 ? RewriteKeys{52, 12}
+                   : RewriteKeys{0, 0};
+}
+static_assert(rewrite_keys(0).count + rewrite_keys(1).count + rewrite_keys(2).count + rewrite_keys(3).count +
+                      rewrite_keys(4).count + rewrite_keys(5).count + rewrite_keys(6).count +
+                      rewrite_keys(7).count == kPage &&
+                  rewrite_keys(5).first + rewrite_keys(5).count == kPage,
+              "the rewriting warps cover the 64 keys once");
 constexpr int kThreads = 32 * (kWarpGather0 + kGatherWarps);
 
 struct StageInfo {
@@ -149,7 +158,7 @@ struct Bars {
   uint64_t* kv_empty;   // [stage] PV of the stage's tile completed (commit)
   uint64_t* p_full;     // [stage] P of the stage's tile written (4 softmax warps)
   uint64_t* qk_done;    // [stage] both QK^T passes of the stage's tile completed (commit)
-  uint64_t* v_ready;    // [stage] V' of the stage's tile written (4 rewriting gather warps)
+  uint64_t* v_ready;    // [stage] V' of the stage's tile written (6 rewriting gather warps)
   uint64_t* slot_full;  // [slot] a part of QK^T completed into the slot (commit)
   uint64_t* slot_empty; // [slot] the slot was read (4 softmax warps)
   uint64_t* q_full;     // query tile of the next segment in TMEM (4 softmax warps)
@@ -265,14 +274,16 @@ __device__ __forceinline__ void q_prefetch_role(const DecodeParams& p, const Par
 // f16 (exact), RoPE as bf16 (copied), the four scales per key, each warp's
 // largest |scale| per group and its valid-key mask.  Warp gw owns keys
 // [8 gw, 8 gw + 8); lane l (< 8) resolves key 8 gw + l (index -> block table
-// -> row).  While tile t converts, the rows of tile t+1 are warmed in L2, the
-// table entries of tile t+2 and the indices of tile t+3 are in flight.  Lane
+// -> row).  While tile t converts, the table entries of tile t+2 and the
+// indices of tile t+3 are in flight (the rows are not warmed in L2 ahead:
+// that measured no faster).  Lane
 // l converts codes [8 l, 8 l + 8) and [256 + 8 l, 256 + 8 l + 8) and, for
 // l < 16, copies RoPE dims [512 + 4 l, +4) of each of the warp's 8 rows.
 // After converting tile t the rewriting warps rewrite tile t-1 as V' (they
-// wait for its QK^T to complete): lane l of rewriter rw scales key
-// 16 rw + 8 h + l / 4, group l % 4 (128 codes, 16 x 16 B), h = 0, 1, by its
-// scale x 2^-E_g.  So PV of tile t-1 can run while tile t+1
+// wait for its QK^T to complete): lane l of a warp that rewrites keys
+// [first, first + count) scales key first + 8 h + l / 4 (h = 0, 1, while
+// below first + count), group l % 4 (128 codes, 16 x 16 B), by its scale x
+// 2^-E_g.  So PV of tile t-1 can run while tile t+1
 // converts, and the stage it frees is the one tile t+2 needs.
 __device__ __forceinline__ void gather_role(const DecodeParams& p, const Partition& part, uint8_t* smem, Bars bars,
                                             volatile int* abort_flag, int gw) {
@@ -322,7 +333,8 @@ __device__ __forceinline__ void gather_role(const DecodeParams& p, const Partiti
   };
 
   // V' of tile tr (cursor rwc), one tile behind the conversion
-  const int rw = rewrite_index(gw);
+  const RewriteKeys rwk = rewrite_keys(gw);
+  const bool rewriter = rwk.count > 0;
   Cursor rwc = cursor_begin(p, part);
   int tr = 0, rw_seg = -1;
   GroupExp gexp;
@@ -340,7 +352,8 @@ __device__ __forceinline__ void gather_role(const DecodeParams& p, const Partiti
     const float gsc = pow2i(-gexp.e(qq));
 #pragma unroll 1
     for (int h = 0; h < 2; ++h) {
-      const int k = 16 * rw + 8 * h + e;
+      if (8 * h + e >= rwk.count) continue;
+      const int k = rwk.first + 8 * h + e;
       const float f32 = scales[scale_index(s, qq, k)] * gsc;
       const uint32_t f = pack_f16x2(f32, f32);
       uint8_t* row = stage_ptr(smem, s) + k * 128;
@@ -381,20 +394,13 @@ __device__ __forceinline__ void gather_role(const DecodeParams& p, const Partiti
     const int s = t % kStages;
     int phys_n = -1;
     const bool valid_n = finish_resolve(nxt, pend_n, phys_n);
-    if (valid_n) {
-      const uintptr_t a = reinterpret_cast<uintptr_t>(row_ptr(phys_n, pos_n));
-      const uintptr_t first = a >> 7, last = (a + kFp8Row - 1) >> 7;
-      const uintptr_t g = static_cast<uintptr_t>(lane >> 3);
-      if (first + g <= last) prefetch_line_l2(reinterpret_cast<const void*>((first + g) << 7));
-      if (first + g + 4 <= last) prefetch_line_l2(reinterpret_cast<const void*>((first + g + 4) << 7));
-    }
     const Pending pend_nn = start_resolve(nxt2, pos_nn);
     Cursor nxt3 = nxt2;
     cursor_next(p, part, nxt3);
     const int pos_nnn = fetch_pos(nxt3);
     float gm0 = 0.f, gm1 = 0.f;   // lanes < 16: groups 0, 2; lanes >= 16: groups 1, 3
     {
-      // the tile's rows (warmed in L2 a tile ago) are loaded before the
+      // the tile's rows are loaded before the
       // stage is free, so their latency overlaps the wait
       uint2 n0[8], n1[8], rp[8];
       float s0[8], s1[8];
@@ -470,9 +476,9 @@ __device__ __forceinline__ void gather_role(const DecodeParams& p, const Partiti
     pend_n = pend_nn;
     pos_nn = pos_nnn;
     ++t;
-    if (rw >= 0 && t - tr > 1 && !rewrite()) { ok = false; break; }
+    if (rewriter && t - tr > 1 && !rewrite()) { ok = false; break; }
   }
-  while (ok && rw >= 0 && rwc.valid) {
+  while (ok && rewriter && rwc.valid) {
     if (!rewrite()) ok = false;
   }
   if (!ok && lane == 0) raise_abort(abort_flag, p.err);

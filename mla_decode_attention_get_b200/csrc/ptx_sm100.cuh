@@ -168,11 +168,6 @@ __device__ __forceinline__ int ld_nc_s32_if(const int* ptr, bool pred, int fallb
   return v;
 }
 
-// One 128-B line into L2 (fire and forget, through the load/store unit).
-__device__ __forceinline__ void prefetch_line_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
-}
-
 // Warm L2 with `bytes` (multiple of 16) starting at a 16-B aligned address.
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)

@@ -44,7 +44,7 @@ WARPS = 4            # softmax warps, one per TMEM lane quadrant
 GATHER_WARPS = 8     # FP8 kernel
 FP8_PARTS = 5        # FP8 kernel: QK^T parts per tile (latent groups 0-3, RoPE)
 FP8_SLOTS = 3        # FP8 kernel: partial-S slots in TMEM
-FP8_REWRITERS = (0, 1, 4, 5)   # FP8 kernel: the gather warps that rewrite V'
+FP8_REWRITERS = (0, 1, 2, 4, 5, 6)   # FP8 kernel: the gather warps that rewrite V'
 
 
 class ProtocolError(AssertionError):
