@@ -34,7 +34,7 @@
 //  * Warp 0 warms L2 with the next segment's query tile; warp 1 issues the
 //    MMAs; warps 2-5 stage the query tile in TMEM, run the softmax and the
 //    epilogue; warps 6-13 gather and convert the cache rows of each 64-key
-//    tile into a three-stage ring, and rewrite V' one tile behind.
+//    tile into a three-stage ring, and six of them rewrite V' one tile behind.
 //  * A stage holds 9 swizzled 64-key x 64-dim chunks (8 of f16 codes, 1 of
 //    bf16 RoPE); the RoPE chunk holds the tile's P (f16) once QK^T of the
 //    tile has completed.
@@ -668,8 +668,8 @@ __device__ __forceinline__ float write_q_tile(const DecodeParams& p, const UnitI
 }
 
 // ---------------------------------------------------------------------------
-// Warps 2-5: per tile, the logits from the partial sums, the online softmax,
-// the P' tiles; per segment, the epilogue.
+// Warps 2-5: per tile, the logits from the partial sums, the online softmax
+// and P; per segment, the epilogue.
 __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partition& part, uint8_t* smem, Bars bars,
                                              uint32_t tmem_base, volatile int* abort_flag) {
   const int lane = threadIdx.x & 31;
