@@ -316,17 +316,19 @@ class Model:
 # The FP8 kernel (`csrc/decode_fp8_sm100.cu`) has its own protocol:
 # - three stages, converted by 8 gather warps (kv_full) and freed by the
 #   commit after PV of their tile (kv_empty);
-# - QK^T in two passes per tile into three TMEM buffers: pass A (groups 0-2,
-#   committed to sa_full) once the tile is in, the query tile is loaded and the
-#   softmax has read pass B of the previous tile (sb_empty); pass B (group 3
-#   and RoPE into buffers 0-1, committed to sb_full and to the stage's qk_done)
-#   once the softmax has read pass A (sa_empty);
-# - the softmax writes the tile's P into the stage's RoPE chunk (which pass B
-#   reads) after pass B has completed, and arrives p_full;
-# - after converting tile t the gather warps rewrite the codes of tile t-1 as
-#   V' (waiting on qk_done: QK^T reads the codes) and arrive v_ready;
-# - the MMA warp issues, in order per tile: pass A(t), pass B(t), PV(t-1), and
-#   PV(t) at the end of a segment; PV waits p_full and v_ready.
+# - QK^T in five parts per tile (latent groups 0-3, RoPE), part i of tile t
+#   being item n = 5 t + i of a ring of three TMEM slots: the MMA warp writes
+#   slot n % 3 once the four softmax warps have read its previous item
+#   (slot_empty) and commits slot_full; the first part also waits for the
+#   tile (kv_full) and, at a segment's start, the query tile (q_full); the
+#   last commits the stage's qk_done as well;
+# - the softmax writes the tile's P into the stage's RoPE chunk (which the
+#   RoPE part reads) after that part has completed, and arrives p_full;
+# - after converting tile t, the six rewriting gather warps rewrite the codes
+#   of tile t-1 as V' (waiting on qk_done: QK^T reads the codes) and arrive
+#   v_ready;
+# - the MMA warp issues, in order per tile: the five parts of QK^T(t),
+#   PV(t-1), and PV(t) at the end of a segment; PV waits p_full and v_ready.
 FP8_STAGES = 3
 
 
