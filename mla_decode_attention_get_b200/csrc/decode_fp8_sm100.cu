@@ -733,9 +733,9 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
                              (static_cast<uint32_t>(info[s].mask[4 * half + 3]) << 24);
       const float4 gmax = GroupExp::tile_max(info[s]);
       const float* sck = scales + scale_index(s, 0, key0);   // group g of this half's keys: sck[g * kPage + i]
-      const float f = rho * scale_log2;
       // the five parts of QK^T, each from its ring slot:
-      //   x = (sum_g scale[k][g] * S_g) * 2^e_r * scale_log2 + S_rope * scale_log2
+      //   x = (sum_g scale[k][g] * S_g) * 2^e_r + S_rope  (= q.k; the softmax
+      //   scale enters with the row max and the exponent)
       float x[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) x[i] = 0.f;
@@ -768,7 +768,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
             }
           } else {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) x[q] = x[q] * f + y[q] * scale_log2;
+            for (int q = 0; q < 32; ++q) x[q] = fmaf(x[q], rho, y[q]);
           }
         }
         if (lane == 0 && q4 == 2 && i == 2) FP8_TRACE(7, t);
@@ -783,8 +783,10 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
           const int nc = min(max(lim - kPage * j - key0, 0), 32);
           m &= nc >= 32 ? 0xFFFFFFFFu : ((1u << nc) - 1u);
         }
+        if (m != 0xFFFFFFFFu) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[i] = ((m >> i) & 1u) ? x[i] : -INFINITY;
+          for (int i = 0; i < 32; ++i) x[i] = ((m >> i) & 1u) ? x[i] : -INFINITY;
+        }
         // pairwise, so that the chain is five deep instead of 32
         float mx[16];
 #pragma unroll
@@ -794,7 +796,7 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
 #pragma unroll
           for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
         }
-        tmax = mx[0];
+        tmax = mx[0] * scale_log2;   // log2 units (scale_log2 > 0 keeps the max)
       }
       tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
       const bool need = tmax > m_run + kRescaleThreshold;
@@ -843,8 +845,8 @@ __device__ __forceinline__ void softmax_role(const DecodeParams& p, const Partit
           float ps[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float a = fast_exp2(x[2 * i] - m_safe);
-            const float b = fast_exp2(x[2 * i + 1] - m_safe);
+            const float a = fast_exp2(fmaf(x[2 * i], scale_log2, -m_safe));
+            const float b = fast_exp2(fmaf(x[2 * i + 1], scale_log2, -m_safe));
             ps[i] = a + b;
             pk[i] = pack_f16x2(a, b);
           }
