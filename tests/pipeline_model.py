@@ -341,7 +341,10 @@ class Fp8Model:
     - "early_p": the softmax writes P before the RoPE part of QK^T (the last
       reader of the chunk P goes to) has completed;
     - "early_v": the gather rewrites V' without waiting for qk_done;
-    - "no_seg_end_pv": PV of a segment's last tile waits for the next tile."""
+    - "no_seg_end_pv": PV of a segment's last tile waits for the next tile
+      (a deadlock only while the ring has fewer slots than a tile has parts);
+    - "early_q": the softmax stages the next segment's query tile before the
+      QK^T parts of the segment's last tile have completed."""
 
     def __init__(self, plan: Plan, seed: int, mutation: Optional[str] = None):
         self.plan, self.rng, self.mut = plan, random.Random(seed), mutation
@@ -470,6 +473,10 @@ class Fp8Model:
                 s = t % FP8_STAGES
                 yield ("wait", lambda s=s, t=t: self.kv_full[s].passes(t // FP8_STAGES))
                 wrote_p = False
+                staged_q = False
+                if self.mut == "early_q" and j == n - 1 and k + 1 < len(self.plan.segments):
+                    yield from self._stage_next_q(w, t, k)
+                    staged_q = True
                 for i in range(FP8_PARTS):
                     if i == FP8_PARTS - 1 and self.mut == "early_p" and live:
                         yield from self._write_p(w, t, s)
@@ -498,12 +505,8 @@ class Fp8Model:
                 self.p_full[s].arrive(t // FP8_STAGES)
                 any_pv = True
                 if j == n - 1:
-                    if k + 1 < len(self.plan.segments):
-                        if t not in self.qk_all_done:
-                            raise ProtocolError(f"softmax {w} overwrites the query tile while QK of tile {t} runs")
-                        self._stage_q(k + 1)
-                        yield ("step",)
-                        self.q_full.arrive(k + 1)
+                    if k + 1 < len(self.plan.segments) and not staged_q:
+                        yield from self._stage_next_q(w, t, k)
                     if live:
                         yield ("wait", lambda s=s, t=t: self.kv_empty[s].passes(t // FP8_STAGES))
                         if t not in self.pv_done:
@@ -513,6 +516,13 @@ class Fp8Model:
                         self.o_busy.discard(w)
                     self.epilogue_done[k] = self.epilogue_done.get(k, 0) + 1
                 t += 1
+
+    def _stage_next_q(self, w, t, k):
+        if t not in self.qk_all_done:
+            raise ProtocolError(f"softmax {w} overwrites the query tile while QK of tile {t} runs")
+        self._stage_q(k + 1)
+        yield ("step",)
+        self.q_full.arrive(k + 1)
 
     def _stage_q(self, seg):
         self.q_writes[seg] = self.q_writes.get(seg, 0) + 1

@@ -48,7 +48,7 @@ def test_fp8_protocol_runs_clean_on_random_schedules():
         PM.Fp8Model(PM.Plan([1, 1, 1, 1, 1], 4, True, {}), seed).run()
 
 
-@pytest.mark.parametrize("mutation", ["no_slot_wait", "early_p", "early_v", "no_seg_end_pv"])
+@pytest.mark.parametrize("mutation", ["no_slot_wait", "early_p", "early_v", "no_seg_end_pv", "early_q"])
 def test_fp8_planted_mistakes_are_caught(mutation):
     caught = 0
     for seed in range(60):
