@@ -108,6 +108,19 @@ def test_sparse_prefill_shape():
     assert_close(out, lse, *oracle(w))
 
 
+@pytest.mark.parametrize("topk", [64, 100])
+@pytest.mark.parametrize("h_q", [16, 64, 128])
+def test_sparse_head_counts_and_topk(h_q, topk):
+    # one or two 64-row tiles per token, a whole or a partial last key tile,
+    # and a token whose list repeats an index (each copy counts as a key)
+    w = I.make_workload(f"sphk{h_q}_{topk}", 2, 2, h_q, [3000, 130], fp8=True, topk=topk, seed=60 + h_q + topk,
+                        pad_rows_per_token=7, num_padded_rows=1)
+    w.indices[1, 0, 3] = w.indices[1, 0, 2]
+    out, lse, err = run(w)
+    assert err == 0
+    assert_close(out, lse, *oracle(w))
+
+
 @pytest.mark.parametrize("parts", [1, 3, 148])
 def test_sparse_output_independent_of_partition_count(parts):
     w = I.make_workload("sp", 3, 2, 32, [4000, 700, 90], fp8=True, topk=300, seed=5,
