@@ -1040,7 +1040,30 @@ cudaError_t launch_decode_fp8(const DecodeParams& p, int row_tiles, cudaStream_t
     if (e != cudaSuccess) return e;
     __atomic_fetch_or(&configured, bit, __ATOMIC_RELEASE);
   }
-  return launch_dependent(mla_decode_fp8_kernel, dim3(p.num_parts, row_tiles), dim3(kThreads), smem, stream, p);
+  // The row tiles of a partition read the same rows: as one cluster they
+  // share a GPC and its side of L2.  Only when every cluster fits at once.
+  static int fits[64] = {};
+  unsigned cy = 1;
+  if (row_tiles == 2 && dev >= 0 && dev < 64) {
+    if (fits[dev] == 0) {
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(p.num_parts, row_tiles);
+      q.blockDim = dim3(kThreads);
+      q.dynamicSmemBytes = smem;
+      cudaLaunchAttribute a[1];
+      a[0].id = cudaLaunchAttributeClusterDimension;
+      a[0].val.clusterDim.x = 1;
+      a[0].val.clusterDim.y = 2;
+      a[0].val.clusterDim.z = 1;
+      q.attrs = a;
+      q.numAttrs = 1;
+      int clusters = 0;
+      fits[dev] = (cudaOccupancyMaxActiveClusters(&clusters, mla_decode_fp8_kernel, &q) == cudaSuccess) ? clusters : -1;
+    }
+    if (fits[dev] >= p.num_parts) cy = 2;
+  }
+  return launch_dependent_cluster(mla_decode_fp8_kernel, dim3(p.num_parts, row_tiles), dim3(kThreads), smem, cy,
+                                  stream, p);
 }
 
 }  // namespace mla
