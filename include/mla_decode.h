@@ -145,11 +145,15 @@ typedef struct mla_decode_args {
   int32_t is_fp8;               /* k_cache holds FP8 rows: read through indices
                                    (sparse) or, with indices == NULL, walked page
                                    by page like the bf16 cache (dense; causal
-                                   applies).  The FP8 path dequantises into f16
-                                   and runs its
-                                   products on f16 operands (fp32 accumulation):
-                                   dequantised cache values and q must lie
-                                   within +-65504, the f16 range. */
+                                   applies).  The logits carry no dequantisation
+                                   rounding: codes enter the MMA as exact f16,
+                                   each 128-value group keeps its own fp32 sum,
+                                   the fp32 scales multiply the sums, and q is
+                                   scaled per row by a power of two into the f16
+                                   range, so any finite scale and any bf16 q are
+                                   accepted.  V enters PV as f16 code x scale
+                                   (x a per-group power of two), which rounds
+                                   only the output. */
 } mla_decode_args;
 
 /*
