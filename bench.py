@@ -275,7 +275,7 @@ def bench_sparse_prefill(args) -> int:
     print(json.dumps({
         "metric": "sparse prefill TFLOP/s (2*(576+512) FLOPs per (row, valid index))", "value": round(tfs, 1),
         "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
-        "higher_is_better": True, "dtype": "f16 (FP8 cache dequantised)", "data": "synthetic",
+        "higher_is_better": True, "dtype": "f16 (exact e4m3 codes; fp32 scales after the MMA)", "data": "synthetic",
         "config": {"workload": w.name, "flops": flops, "kv_bytes": kv_bytes},
         "roofline": {"bound": "tensor", "achieved": round(tfs, 1), "peak": tc_sus, "unit": "TFLOP/s",
                      "frac": round(tfs / tc_sus, 4), "peak_kind": "sustained bf16 GEMM",
