@@ -85,6 +85,11 @@ constexpr int kStages = 3;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemQCol = 128;           // Q tile columns 128..415 in lanes 16-31
 constexpr int kPChunk = kChunks - 1;          // the RoPE chunk of a stage, reused for the page's P tile
+// A stage is refilled in two parts: its chunks 0-3 (dims 0-255), which only
+// QK^T and the first half of PV read, as soon as that half has completed,
+// and chunks 4-8 (dims 256-575, P in chunk 8) once all of PV has.
+constexpr int kLoChunks = 4;
+static_assert(kLoChunks < kPChunk, "P lives in the part released last");
 
 constexpr int kWarpLoad = 0, kWarpMma = 1, kWarpEnd = 6;   // warps 2-5: softmax
 constexpr int kThreads = 32 * kWarpEnd;
@@ -94,8 +99,9 @@ struct Smem {
   // its P tile ([64 rows x 64 keys], the same 128-B swizzled geometry)
   static constexpr int kv_off = 0;
   static constexpr int bar_off = kv_off + kStages * kPageBytes;
-  // kv_full[S], kv_empty[S], s_full[2], s_empty[2], q_full, p_full[S], done
-  static constexpr int n_bars = 3 * kStages + 6;
+  // kv_full[S], kv_empty_lo[S], s_full[2], s_empty[2], q_full, p_full[S],
+  // done, kv_empty[S]
+  static constexpr int n_bars = 4 * kStages + 6;
   static constexpr int info_off = bar_off + n_bars * 8;
   static constexpr int info_bytes = kStages * 16;                // per stage: valid keys of the page
   static constexpr int misc_off = info_off + info_bytes;         // tmem base, abort flag
@@ -111,8 +117,9 @@ struct StageInfo {
 };
 
 struct Bars {
-  uint64_t* kv_full;
-  uint64_t* kv_empty;
+  uint64_t* kv_full;      // per stage: both parts of the page landed (two arrivals)
+  uint64_t* kv_empty_lo;  // per stage: chunks 0-3 free (first half of PV completed)
+  uint64_t* kv_empty;     // per stage: the whole stage free (PV completed)
   uint64_t* s_full;
   uint64_t* s_empty;
   uint64_t* q_full;
@@ -149,9 +156,10 @@ struct Issued {
 static_assert(kStages == 3, "Issued holds three stages");
 
 // ---------------------------------------------------------------------------
-// Warp 0 (one lane): TMA loads of cache pages, their block-table entries
-// read kPrefetchPages pages ahead, and an L2 prefetch of the next segment's
-// query tile.  (Warming the pages themselves in L2 ahead of their loads, 1 to
+// Warp 0 (one lane): TMA loads of cache pages, each in two parts (chunks 0-3
+// once the stage's first PV half has completed, chunks 4-8 once all of PV
+// has), their block-table entries read kPrefetchPages pages ahead, and an L2
+// prefetch of the next segment's query tile.  (Warming the pages themselves in L2 ahead of their loads, 1 to
 // 4 pages ahead, measured slower than not warming them at all.)
 __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition& part, const CUtensorMap* tmap_kv,
                                           uint8_t* smem, Bars bars, StageInfo* info, volatile int* abort_flag,
@@ -161,9 +169,9 @@ __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition
   int t = 0;
   bool ok = true;
 
-  // Physical pages of the next kPrefetchPages pages, read when they are
-  // warmed in L2 so that a page's TMA load never waits on the block table
-  // (four scalars: an indexed array would live in local memory).
+  // Physical pages of the next kPrefetchPages pages, read ahead so that a
+  // page's TMA load never waits on the block table (four scalars: an indexed
+  // array would live in local memory).
   static_assert(kPrefetchPages == 4, "the page ring holds four entries");
   int r0 = -1, r1 = -1, r2 = -1, r3 = -1;
   auto ring_set = [&](int j, int phys) {
@@ -189,7 +197,8 @@ __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition
       for (int j = jb; j < jn; ++j) ring_set(j, page_of(p, ui.b, j));
       for (int j = jb; j < je; ++j) {
         const int s = t % kStages;
-        if (!mbar_wait(&bars.kv_empty[s], ((t / kStages) & 1) ^ 1, abort_flag, p.wait_ns)) { ok = false; return false; }
+        const uint32_t free_parity = ((t / kStages) & 1) ^ 1;
+        if (!mbar_wait(&bars.kv_empty_lo[s], free_parity, abort_flag, p.wait_ns)) { ok = false; return false; }
         MLA_TRACE_EV(0, t);
         int nv = min(kPage, ui.L - kPage * j);
         const int phys = ring_get(j);
@@ -197,14 +206,32 @@ __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition
           atomicOr(p.err, kErrBlockTable);
           nv = 0;
         }
+        // (the stage's previous page is done with its info: the MMA warp read
+        // it before QK^T, the softmax before writing the P that PV read)
         info[s].nvalid = nv;
+        uint8_t* dst = smem + Smem::kv_off + s * kPageBytes;
+        // kv_full takes two arrivals per page, one per part
         if (nv > 0) {
-          mbar_arrive_expect_tx(&bars.kv_full[s], kPageBytes);
-          uint8_t* dst = smem + Smem::kv_off + s * kPageBytes;
+          mbar_arrive_expect_tx(&bars.kv_full[s], kLoChunks * kChunkBytes);
 #pragma unroll 1
-          for (int c = 0; c < kChunks; ++c)
+          for (int c = 0; c < kLoChunks; ++c)
             tma_load_3d(dst + c * kChunkBytes, tmap_kv, &bars.kv_full[s], 64 * c, 0, phys, pol_kv);
           issued.set(s, t);
+        } else {
+          mbar_arrive(&bars.kv_full[s]);
+        }
+        if (!mbar_wait(&bars.kv_empty[s], free_parity, abort_flag, p.wait_ns)) {
+          // the page's second arrival, so that the drain at exit sees its
+          // first part land
+          mbar_arrive(&bars.kv_full[s]);
+          ok = false;
+          return false;
+        }
+        if (nv > 0) {
+          mbar_arrive_expect_tx(&bars.kv_full[s], (kChunks - kLoChunks) * kChunkBytes);
+#pragma unroll 1
+          for (int c = kLoChunks; c < kChunks; ++c)
+            tma_load_3d(dst + c * kChunkBytes, tmap_kv, &bars.kv_full[s], 64 * c, 0, phys, pol_kv);
         } else {
           mbar_arrive(&bars.kv_full[s]);
         }
@@ -265,6 +292,7 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
         const bool acc0 = (o_seg == pv.seg);
         const uint64_t vd = v_desc0 + ((s * kPageBytes) >> 4);
         const uint64_t pd = p_desc0 + ((s * kPageBytes) >> 4);
+        static_assert(kLoChunks == 4, "the first PV half reads chunks 0-3");
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
 #pragma unroll
@@ -272,8 +300,13 @@ __device__ __forceinline__ void mma_role(const DecodeParams& p, const Partition&
             umma_bf16_elect(tmem_base + h * 256, pd + ((k * 32) >> 4),
                             vd + ((4 * h * kChunkBytes + k * 2048) >> 4), idesc_pv, (acc0 || k > 0) ? 1u : 0u);
           }
+          // chunks 0-3 of the stage are free once the first half (and QK^T,
+          // issued before it) has completed
+          if (h == 0) umma_commit_elect(&bars.kv_empty_lo[s]);
         }
         o_seg = pv.seg;
+      } else {
+        umma_commit_elect(&bars.kv_empty_lo[s]);
       }
       // the stage (K, V and P of the page) is free once PV has completed
       umma_commit_elect(&bars.kv_empty[s]);
@@ -583,12 +616,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Smem::bar_off);
   Bars bars;
   bars.kv_full = bar;
-  bars.kv_empty = bar + kStages;
+  bars.kv_empty_lo = bar + kStages;
   bars.s_full = bar + 2 * kStages;
   bars.s_empty = bar + 2 * kStages + 2;
   bars.q_full = bar + 2 * kStages + 4;
   bars.p_full = bar + 2 * kStages + 5;
   bars.done = bar + 3 * kStages + 5;
+  bars.kv_empty = bar + 3 * kStages + 6;
   StageInfo* info = reinterpret_cast<StageInfo*>(smem + Smem::info_off);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::misc_off);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::misc_off + 4);
@@ -597,7 +631,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     *abort_flag = misaligned ? 1 : 0;
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars.kv_full[s], 1);
+      mbar_init(&bars.kv_full[s], 2);
+      mbar_init(&bars.kv_empty_lo[s], 1);
       mbar_init(&bars.kv_empty[s], 1);
       mbar_init(&bars.p_full[s], 4);
       info[s].nvalid = 0;

@@ -7,7 +7,10 @@ hand-offs of one CTA of the bf16 decode kernel in `csrc/decode_sm100.cu`:
 - the four softmax warps, with idle padding warps, lazy rescales, segment
   epilogues and query-tile staging.
 A random scheduler then interleaves the roles, the landing of page loads and
-the in-order completion of the tensor pipe.
+the in-order completion of the tensor pipe.  A page is loaded in two parts:
+chunks 0-3 (dims 0-255; QK^T and the first PV half read them) once the first
+PV half of the stage's previous page has completed (kv_empty_lo), chunks 4-8
+once all of its PV has (kv_empty); kv_full takes one arrival per part.
 
 An mbarrier is modelled by its count, its pending arrivals and the number of
 phases it has completed.  A wait on parity P passes when the completed count
@@ -26,7 +29,11 @@ catch it:
 - "shared_p_full": one p_full barrier for all pages;
 - "no_rescale_wait": rescale O without waiting for PV of the previous page;
 - "single_pv_barrier": the epilogue waits for PV through one barrier
-  committed per page, with parity t & 1.
+  committed per page, with parity t & 1;
+- "hi_on_lo": the second part of a page (chunks 4-8, P in chunk 8) is loaded
+  once the first PV half has completed, like the first part;
+- "lo_before_pv": the first part's release is committed before the first PV
+  half is issued.
 
 `Fp8Model` (at the end) does the same for the FP8 kernel in
 `csrc/decode_fp8_sm100.cu`, whose protocol differs (three stages filled by 8
@@ -83,6 +90,8 @@ class Plan:
 @dataclass
 class State:
     stage_page: List[Optional[int]] = field(default_factory=lambda: [None] * STAGES)
+    stage_page_lo: List[Optional[int]] = field(default_factory=lambda: [None] * STAGES)   # bf16: chunks 0-3
+    pv_lo_done: set = field(default_factory=set)                                         # bf16: first PV half
     stage_writers: List[int] = field(default_factory=lambda: [0] * STAGES)
     qk_done: set = field(default_factory=set)
     pv_done: set = field(default_factory=set)
@@ -106,7 +115,8 @@ class Model:
             self.seg_of += [k] * n
             t += n
         S = STAGES
-        self.kv_full = [Barrier(f"kv_full[{s}]", 1) for s in range(S)]
+        self.kv_full = [Barrier(f"kv_full[{s}]", 2) for s in range(S)]
+        self.kv_empty_lo = [Barrier(f"kv_empty_lo[{s}]", 1) for s in range(S)]
         self.kv_empty = [Barrier(f"kv_empty[{s}]", 1) for s in range(S)]
         self.s_full = [Barrier(f"s_full[{b}]", 1) for b in range(2)]
         self.s_empty = [Barrier(f"s_empty[{b}]", WARPS) for b in range(2)]
@@ -119,7 +129,7 @@ class Model:
         self.pv_bar = Barrier("pv_done", 1)          # only the planted mistake waits on it
         self.st = State()
         self.pipe: List[tuple] = []                  # tensor pipe, in order
-        self.loads: List[int] = []                   # pages in flight (bf16 path)
+        self.loads: List[tuple] = []                 # (page, part) in flight; part 0: chunks 0-3
 
     # -- phase bookkeeping ---------------------------------------------------
     def p_full_phase(self, t):
@@ -129,9 +139,14 @@ class Model:
     def producer(self):
         for t in range(self.T):
             s = t % STAGES
-            yield ("wait", lambda s=s, t=t: self.kv_empty[s].passes(t // STAGES - 1))
-            self._stage_write_begin(s, t)
-            self.loads.append(t)
+            yield ("wait", lambda s=s, t=t: self.kv_empty_lo[s].passes(t // STAGES - 1))
+            self._stage_write_begin(s, t, 0)
+            self.loads.append((t, 0))
+            yield ("step",)
+            second = self.kv_empty_lo if self.mut == "hi_on_lo" else self.kv_empty
+            yield ("wait", lambda s=s, t=t: second[s].passes(t // STAGES - 1))
+            self._stage_write_begin(s, t, 1)
+            self.loads.append((t, 1))
             yield ("step",)
 
     def mma(self):
@@ -141,7 +156,13 @@ class Model:
             issued = False
             if pv < qk and self.p_full[pv % STAGES].passes(self.p_full_phase(pv)):
                 s = pv % STAGES
-                self.pipe.append(("PV", pv, self.seg_of[pv] != o_seg))
+                first = self.seg_of[pv] != o_seg
+                if self.mut == "lo_before_pv":
+                    self.pipe.append(("commit", self.kv_empty_lo[s], pv // STAGES))
+                self.pipe.append(("PV", pv, first, 0))
+                if self.mut != "lo_before_pv":
+                    self.pipe.append(("commit", self.kv_empty_lo[s], pv // STAGES))
+                self.pipe.append(("PV", pv, first, 1))
                 o_seg = self.seg_of[pv]
                 self.pipe.append(("commit", self.kv_empty[s], pv // STAGES))
                 if self.mut == "single_pv_barrier":
@@ -216,19 +237,28 @@ class Model:
                 t += 1
 
     # -- helpers ---------------------------------------------------------------
-    def _stage_write_begin(self, s, t):
-        prev = self.st.stage_page[s]
-        if prev is not None and prev != t and prev not in self.st.pv_done:
-            raise ProtocolError(f"page {t} overwrites stage {s} while page {prev} is still in use")
+    def _stage_write_begin(self, s, t, part=None):
+        """part: None for a whole stage (FP8 model), 0 or 1 for the bf16
+        model's chunks 0-3 or 4-8."""
+        if part == 0:
+            prev, done = self.st.stage_page_lo[s], self.st.pv_lo_done
+        else:
+            prev, done = self.st.stage_page[s], self.st.pv_done
+        if prev is not None and prev != t and prev not in done:
+            where = "" if part is None else f" (part {part})"
+            raise ProtocolError(f"page {t} overwrites stage {s}{where} while page {prev} is still in use")
 
     def _stage_q(self, w, seg):
         self.st.q_writes[seg] = self.st.q_writes.get(seg, 0) + 1
         if self.st.q_writes[seg] == WARPS:
             self.st.q_seg = seg
 
-    def _land(self, t):
+    def _land(self, t, part):
         s = t % STAGES
-        self.st.stage_page[s] = t
+        if part == 0:
+            self.st.stage_page_lo[s] = t
+        else:
+            self.st.stage_page[s] = t
         self.kv_full[s].arrive(t // STAGES)
 
     def _pipe_pop(self):
@@ -239,8 +269,9 @@ class Model:
         elif kind == "QK":
             t = item[1]
             s, sb = t % STAGES, t & 1
-            if self.st.stage_page[s] != t:
-                raise ProtocolError(f"QK of page {t} reads stage {s} holding {self.st.stage_page[s]}")
+            if self.st.stage_page[s] != t or self.st.stage_page_lo[s] != t:
+                raise ProtocolError(f"QK of page {t} reads stage {s} holding "
+                                    f"{self.st.stage_page_lo[s]} / {self.st.stage_page[s]}")
             if self.st.q_seg != self.seg_of[t]:
                 raise ProtocolError(f"QK of page {t} reads the query tile of segment {self.st.q_seg}")
             if self.st.s_reading[sb]:
@@ -248,10 +279,12 @@ class Model:
             self.st.s_page[sb] = t
             self.st.qk_done.add(t)
         else:
-            t, first = item[1], item[2]
+            t, first, half = item[1], item[2], item[3]
             s = t % STAGES
-            if self.st.stage_page[s] != t:
-                raise ProtocolError(f"PV of page {t} reads stage {s} holding {self.st.stage_page[s]}")
+            # P lives in chunk 8 (the second part): both halves read it
+            if self.st.stage_page[s] != t or (half == 0 and self.st.stage_page_lo[s] != t):
+                raise ProtocolError(f"PV half {half} of page {t} reads stage {s} holding "
+                                    f"{self.st.stage_page_lo[s]} / {self.st.stage_page[s]}")
             if self.st.p_written.get(t, 0) != self.plan.live_warps:
                 raise ProtocolError(f"PV of page {t} reads P before every live warp wrote it")
             if self.st.o_busy:
@@ -259,7 +292,10 @@ class Model:
             seg = self.seg_of[t]
             if first and seg > 0 and self.st.epilogue_done.get(seg - 1, 0) != WARPS:
                 raise ProtocolError(f"PV of page {t} restarts O before the epilogue of segment {seg - 1}")
-            self.st.pv_done.add(t)
+            if half == 0:
+                self.st.pv_lo_done.add(t)
+            else:
+                self.st.pv_done.add(t)
 
     # -- scheduler -------------------------------------------------------------
     def run(self, max_steps: int = 200000):
@@ -291,7 +327,7 @@ class Model:
                     movers.append(("role", i))
             if self.pipe:
                 movers.append(("pipe", None))
-            movers += [("land", t) for t in self.loads]
+            movers += [("land", x) for x in self.loads]
             if not movers:
                 if not polls:
                     raise ProtocolError("deadlock: no role can move and nothing is in flight")
@@ -308,7 +344,7 @@ class Model:
                 self._pipe_pop()
             else:
                 self.loads.remove(arg)
-                self._land(arg)
+                self._land(*arg)
         raise ProtocolError("no completion within the step budget")
 
 

@@ -3,7 +3,8 @@
 `pipeline_model` restates the hand-offs of one CTA of the bf16 decode kernel
 (and, in `Fp8Model`, of the FP8 kernel, with its five-part QK^T through a
 ring of three TMEM slots and the V' rewrite by the gather warps):
-- the page producer: TMA, or 8 gather warps on the FP8 kernel;
+- the page producer: TMA in two parts per page, or 8 gather warps on the FP8
+  kernel;
 - the MMA warp's event loop;
 - four softmax warps, with padding warps, lazy rescales, segment epilogues and
   query-tile staging.
@@ -60,7 +61,8 @@ def test_fp8_planted_mistakes_are_caught(mutation):
     assert caught > 0
 
 
-@pytest.mark.parametrize("mutation", ["shared_p_full", "no_rescale_wait", "single_pv_barrier"])
+@pytest.mark.parametrize("mutation", ["shared_p_full", "no_rescale_wait", "single_pv_barrier", "hi_on_lo",
+                                      "lo_before_pv"])
 def test_planted_mistakes_are_caught(mutation):
     caught = 0
     for seed in range(60):
