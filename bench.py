@@ -49,8 +49,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # when a kernel changed since or the workload was not captured.  The MTP
 # shapes were captured on 16 of their 132 sequences and scaled by 132 / 16
 # (the same row tiles re-read the same pages of every sequence).
-ATTN_TRAFFIC_BYTES = {"C1": None, "C2": 611676928, "C3": 330269440, "C4": 2577833280, "C5": 119535616,
-                      "MTP s_q=4": 2609166912}
+ATTN_TRAFFIC_BYTES = {"C1": None, "C2": 612192768, "C3": 330257152, "C4": 2572225920, "C5": 119535616,
+                      "MTP s_q=4": 2609194368}
 
 
 def _env_int(k, d):

@@ -7,10 +7,12 @@ hand-offs of one CTA of the bf16 decode kernel in `csrc/decode_sm100.cu`:
 - the four softmax warps, with idle padding warps, lazy rescales, segment
   epilogues and query-tile staging.
 A random scheduler then interleaves the roles, the landing of page loads and
-the in-order completion of the tensor pipe.  A page is loaded in two parts:
-chunks 0-3 (dims 0-255; QK^T and the first PV half read them) once the first
-PV half of the stage's previous page has completed (kv_empty_lo), chunks 4-8
-once all of its PV has (kv_empty); kv_full takes one arrival per part.
+the in-order completion of the tensor pipe.  A page is loaded in `parts`
+parts (REFILL_PARTS): PV runs in as many slices of the 512 value dims, part i
+(of all but the last) holds the chunks only QK^T and PV slice i read and is
+loaded once that slice of the stage's previous page has completed
+(kv_empty_part[i]); the last part (P's chunk included) once all of PV has
+(kv_empty).  kv_full takes one arrival per part.
 
 An mbarrier is modelled by its count, its pending arrivals and the number of
 phases it has completed.  A wait on parity P passes when the completed count
@@ -30,10 +32,10 @@ catch it:
 - "no_rescale_wait": rescale O without waiting for PV of the previous page;
 - "single_pv_barrier": the epilogue waits for PV through one barrier
   committed per page, with parity t & 1;
-- "hi_on_lo": the second part of a page (chunks 4-8, P in chunk 8) is loaded
-  once the first PV half has completed, like the first part;
+- "hi_on_lo": the last part of a page (P's chunk included) is loaded once
+  the PV slice before the last has completed, like the part before it;
 - "lo_before_pv": the first part's release is committed before the first PV
-  half is issued.
+  slice is issued.
 
 `Fp8Model` (at the end) does the same for the FP8 kernel in
 `csrc/decode_fp8_sm100.cu`, whose protocol differs (three stages filled by 8
@@ -47,6 +49,7 @@ from dataclasses import dataclass, field
 from typing import Dict, List, Optional
 
 STAGES = 3
+REFILL_PARTS = 2     # bf16 kernel: parts a stage is refilled in
 WARPS = 4            # softmax warps, one per TMEM lane quadrant
 GATHER_WARPS = 8     # FP8 kernel
 FP8_PARTS = 5        # FP8 kernel: QK^T parts per tile (latent groups 0-3, RoPE)
@@ -90,8 +93,8 @@ class Plan:
 @dataclass
 class State:
     stage_page: List[Optional[int]] = field(default_factory=lambda: [None] * STAGES)
-    stage_page_lo: List[Optional[int]] = field(default_factory=lambda: [None] * STAGES)   # bf16: chunks 0-3
-    pv_lo_done: set = field(default_factory=set)                                         # bf16: first PV half
+    stage_page_part: Dict[int, List[Optional[int]]] = field(default_factory=dict)   # bf16: all but the last part
+    pv_part_done: Dict[int, set] = field(default_factory=dict)                       # bf16: PV slices but the last
     stage_writers: List[int] = field(default_factory=lambda: [0] * STAGES)
     qk_done: set = field(default_factory=set)
     pv_done: set = field(default_factory=set)
@@ -105,8 +108,8 @@ class State:
 
 
 class Model:
-    def __init__(self, plan: Plan, seed: int, mutation: Optional[str] = None):
-        self.plan, self.rng, self.mut = plan, random.Random(seed), mutation
+    def __init__(self, plan: Plan, seed: int, mutation: Optional[str] = None, parts: int = REFILL_PARTS):
+        self.plan, self.rng, self.mut, self.parts = plan, random.Random(seed), mutation, parts
         self.T = sum(plan.segments)
         self.seg_of, self.first_of_seg = [], set()
         t = 0
@@ -115,8 +118,8 @@ class Model:
             self.seg_of += [k] * n
             t += n
         S = STAGES
-        self.kv_full = [Barrier(f"kv_full[{s}]", 2) for s in range(S)]
-        self.kv_empty_lo = [Barrier(f"kv_empty_lo[{s}]", 1) for s in range(S)]
+        self.kv_full = [Barrier(f"kv_full[{s}]", parts) for s in range(S)]
+        self.kv_empty_part = [[Barrier(f"kv_empty_part[{i}][{s}]", 1) for s in range(S)] for i in range(parts - 1)]
         self.kv_empty = [Barrier(f"kv_empty[{s}]", 1) for s in range(S)]
         self.s_full = [Barrier(f"s_full[{b}]", 1) for b in range(2)]
         self.s_empty = [Barrier(f"s_empty[{b}]", WARPS) for b in range(2)]
@@ -128,6 +131,8 @@ class Model:
             self.p_full = [Barrier(f"p_full[{s}]", WARPS) for s in range(S)]
         self.pv_bar = Barrier("pv_done", 1)          # only the planted mistake waits on it
         self.st = State()
+        self.st.stage_page_part = {i: [None] * S for i in range(parts - 1)}
+        self.st.pv_part_done = {i: set() for i in range(parts - 1)}
         self.pipe: List[tuple] = []                  # tensor pipe, in order
         self.loads: List[tuple] = []                 # (page, part) in flight; part 0: chunks 0-3
 
@@ -139,15 +144,16 @@ class Model:
     def producer(self):
         for t in range(self.T):
             s = t % STAGES
-            yield ("wait", lambda s=s, t=t: self.kv_empty_lo[s].passes(t // STAGES - 1))
-            self._stage_write_begin(s, t, 0)
-            self.loads.append((t, 0))
-            yield ("step",)
-            second = self.kv_empty_lo if self.mut == "hi_on_lo" else self.kv_empty
-            yield ("wait", lambda s=s, t=t: second[s].passes(t // STAGES - 1))
-            self._stage_write_begin(s, t, 1)
-            self.loads.append((t, 1))
-            yield ("step",)
+            for i in range(self.parts):
+                last = i == self.parts - 1
+                if last and self.mut == "hi_on_lo":
+                    freed = self.kv_empty_part[i - 1]
+                else:
+                    freed = self.kv_empty if last else self.kv_empty_part[i]
+                yield ("wait", lambda s=s, t=t, freed=freed: freed[s].passes(t // STAGES - 1))
+                self._stage_write_begin(s, t, i)
+                self.loads.append((t, i))
+                yield ("step",)
 
     def mma(self):
         pv = qk = 0
@@ -158,11 +164,11 @@ class Model:
                 s = pv % STAGES
                 first = self.seg_of[pv] != o_seg
                 if self.mut == "lo_before_pv":
-                    self.pipe.append(("commit", self.kv_empty_lo[s], pv // STAGES))
-                self.pipe.append(("PV", pv, first, 0))
-                if self.mut != "lo_before_pv":
-                    self.pipe.append(("commit", self.kv_empty_lo[s], pv // STAGES))
-                self.pipe.append(("PV", pv, first, 1))
+                    self.pipe.append(("commit", self.kv_empty_part[0][s], pv // STAGES))
+                for h in range(self.parts):
+                    self.pipe.append(("PV", pv, first, h))
+                    if h < self.parts - 1 and not (h == 0 and self.mut == "lo_before_pv"):
+                        self.pipe.append(("commit", self.kv_empty_part[h][s], pv // STAGES))
                 o_seg = self.seg_of[pv]
                 self.pipe.append(("commit", self.kv_empty[s], pv // STAGES))
                 if self.mut == "single_pv_barrier":
@@ -237,16 +243,13 @@ class Model:
                 t += 1
 
     # -- helpers ---------------------------------------------------------------
-    def _stage_write_begin(self, s, t, part=None):
-        """part: None for a whole stage (FP8 model), 0 or 1 for the bf16
-        model's chunks 0-3 or 4-8."""
-        if part == 0:
-            prev, done = self.st.stage_page_lo[s], self.st.pv_lo_done
+    def _stage_write_begin(self, s, t, part):
+        if part < self.parts - 1:
+            prev, done = self.st.stage_page_part[part][s], self.st.pv_part_done[part]
         else:
             prev, done = self.st.stage_page[s], self.st.pv_done
         if prev is not None and prev != t and prev not in done:
-            where = "" if part is None else f" (part {part})"
-            raise ProtocolError(f"page {t} overwrites stage {s}{where} while page {prev} is still in use")
+            raise ProtocolError(f"page {t} overwrites stage {s} (part {part}) while page {prev} is still in use")
 
     def _stage_q(self, w, seg):
         self.st.q_writes[seg] = self.st.q_writes.get(seg, 0) + 1
@@ -255,8 +258,8 @@ class Model:
 
     def _land(self, t, part):
         s = t % STAGES
-        if part == 0:
-            self.st.stage_page_lo[s] = t
+        if part < self.parts - 1:
+            self.st.stage_page_part[part][s] = t
         else:
             self.st.stage_page[s] = t
         self.kv_full[s].arrive(t // STAGES)
@@ -269,9 +272,9 @@ class Model:
         elif kind == "QK":
             t = item[1]
             s, sb = t % STAGES, t & 1
-            if self.st.stage_page[s] != t or self.st.stage_page_lo[s] != t:
-                raise ProtocolError(f"QK of page {t} reads stage {s} holding "
-                                    f"{self.st.stage_page_lo[s]} / {self.st.stage_page[s]}")
+            held = [self.st.stage_page_part[i][s] for i in range(self.parts - 1)] + [self.st.stage_page[s]]
+            if any(x != t for x in held):
+                raise ProtocolError(f"QK of page {t} reads stage {s} holding {held}")
             if self.st.q_seg != self.seg_of[t]:
                 raise ProtocolError(f"QK of page {t} reads the query tile of segment {self.st.q_seg}")
             if self.st.s_reading[sb]:
@@ -281,10 +284,10 @@ class Model:
         else:
             t, first, half = item[1], item[2], item[3]
             s = t % STAGES
-            # P lives in chunk 8 (the second part): both halves read it
-            if self.st.stage_page[s] != t or (half == 0 and self.st.stage_page_lo[s] != t):
-                raise ProtocolError(f"PV half {half} of page {t} reads stage {s} holding "
-                                    f"{self.st.stage_page_lo[s]} / {self.st.stage_page[s]}")
+            # P lives in chunk 8 (the last part): every slice reads it
+            own = self.st.stage_page[s] if half == self.parts - 1 else self.st.stage_page_part[half][s]
+            if self.st.stage_page[s] != t or own != t:
+                raise ProtocolError(f"PV slice {half} of page {t} reads stage {s} holding {own} / {self.st.stage_page[s]}")
             if self.st.p_written.get(t, 0) != self.plan.live_warps:
                 raise ProtocolError(f"PV of page {t} reads P before every live warp wrote it")
             if self.st.o_busy:
@@ -292,8 +295,8 @@ class Model:
             seg = self.seg_of[t]
             if first and seg > 0 and self.st.epilogue_done.get(seg - 1, 0) != WARPS:
                 raise ProtocolError(f"PV of page {t} restarts O before the epilogue of segment {seg - 1}")
-            if half == 0:
-                self.st.pv_lo_done.add(t)
+            if half < self.parts - 1:
+                self.st.pv_part_done[half].add(t)
             else:
                 self.st.pv_done.add(t)
 
