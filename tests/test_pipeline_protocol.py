@@ -72,3 +72,27 @@ def test_planted_mistakes_are_caught(mutation):
         except PM.ProtocolError:
             caught += 1
     assert caught > 0
+
+
+def _constants(path):
+    import os
+    import re
+    src = open(os.path.join(os.path.dirname(__file__), "..", "mla_decode_attention_get_b200", "csrc", path)).read()
+    return src, {m.group(1): int(m.group(2)) for m in re.finditer(r"constexpr int (k\w+) = (\d+);", src)}
+
+
+def test_models_mirror_the_kernels():
+    """The models' constants are the kernels' own: a protocol change in the
+    CUDA source that the model does not follow fails here."""
+    import re
+    src, k = _constants("decode_sm100.cu")
+    assert PM.STAGES == k["kStages"]
+    assert re.search(r"mbar_init\(&bars\.kv_full\[s\], %d\)" % PM.REFILL_PARTS, src)
+    assert PM.REFILL_PARTS == 2 and k["kLoChunks"] == 4          # chunks 0-3, then 4-8
+    src8, k8 = _constants("decode_fp8_sm100.cu")
+    assert PM.FP8_STAGES == k8["kStages"]
+    assert PM.FP8_PARTS == k8["kParts"] and PM.FP8_SLOTS == k8["kSlots"]
+    assert PM.GATHER_WARPS == k8["kGatherWarps"]
+    rewriters = sorted(int(gw) for gw, count in re.findall(r"gw == (\d) \? RewriteKeys\{\d+, (\d+)\}", src8)
+                       if int(count) > 0)
+    assert tuple(rewriters) == tuple(sorted(PM.FP8_REWRITERS)) and len(rewriters) == k8["kRewriteWarps"]
