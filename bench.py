@@ -28,6 +28,7 @@ from __future__ import annotations
 
 import argparse
 import gc
+import hashlib
 import json
 import os
 import statistics
@@ -46,11 +47,42 @@ FALLBACK_BF16_TFLOPS = 1590.0
 
 # DRAM traffic (read + write bytes) of one attention-kernel launch per
 # workload, from one ncu capture of the current kernels (profiles/); None
-# when a kernel changed since or the workload was not captured.  The MTP
-# shapes were captured on 16 of their 132 sequences and scaled by 132 / 16
-# (the same row tiles re-read the same pages of every sequence).
+# where the workload was not captured.  The MTP shapes were captured on 16 of
+# their 132 sequences and scaled by 132 / 16 (the same row tiles re-read the
+# same pages of every sequence).
 ATTN_TRAFFIC_BYTES = {"C1": None, "C2": 612192768, "C3": 330257152, "C4": 2572225920, "C5": 119535616,
                       "MTP s_q=4": 2609194368}
+# The sources each attention kernel is built from, and their SHA-256 when the
+# figures above were captured: a kernel whose sources have changed since
+# reports no traffic (null) until it is captured again.
+ATTN_KERNEL_SOURCES = {
+    "mla_decode_kernel": ("decode_sm100.cu", "decode_common.cuh", "ptx_sm100.cuh", "mla_kernels.cuh",
+                          "mla_api.cu"),
+    "mla_decode_fp8_kernel": ("decode_fp8_sm100.cu", "decode_common.cuh", "ptx_sm100.cuh", "mla_kernels.cuh",
+                              "mla_api.cu"),
+}
+ATTN_TRAFFIC_SOURCE_SHA256 = {
+    "mla_decode_kernel": "981accf908896c80338a1b3917dcf53f4876aa1d9f0032097acae137c2649c45",
+    "mla_decode_fp8_kernel": "f1eec4739e0e4722b0ffc0743a1864e3251956a1efe280d46b9c9cdf967d7c52",
+}
+
+
+def kernel_sources_sha256(kernel):
+    h = hashlib.sha256()
+    for name in ATTN_KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "mla_decode_attention_get_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def attn_traffic(key, kernel):
+    """The captured traffic of workload `key`, or None if the kernel's
+    sources differ from those it was captured with."""
+    try:
+        current = kernel_sources_sha256(kernel) == ATTN_TRAFFIC_SOURCE_SHA256[kernel]
+    except OSError:
+        current = False
+    return ATTN_TRAFFIC_BYTES.get(key) if current else None
 
 
 def _env_int(k, d):
@@ -422,7 +454,7 @@ def _gpu_uuid(dev):
 def per_config_record(key, w, tm, ms_step, attn_ms, clocks, peaks, cpu_budget):
     hbm, tc, tc_sus, _ = peaks
     roof = attention_roofline(tm.kv_bytes, tm.flops, attn_ms, hbm, tc, tc_sus)
-    roof["traffic"] = ATTN_TRAFFIC_BYTES.get(key)
+    roof["traffic"] = attn_traffic(key, "mla_decode_fp8_kernel" if w.fp8 else "mla_decode_kernel")
     rec = {
         "workload": _workload_name(key, w), "batch": w.batch, "s_q": w.s_q, "h_q": w.h_q,
         "causal": bool(w.causal), "cache": "fp8" if w.fp8 else "bf16", "topk": w.topk,
@@ -660,7 +692,8 @@ def main():
         return 0
 
     roof = attention_roofline(kv_bytes, flops, attn_ms, hbm, tc, tc_sus)
-    roof.update({"traffic": ATTN_TRAFFIC_BYTES.get(head_key), "peak_source": peak_src,
+    roof.update({"traffic": attn_traffic(head_key, "mla_decode_fp8_kernel" if w.fp8 else "mla_decode_kernel"),
+                 "peak_source": peak_src,
                  "kernel": "mla_decode_fp8_kernel" if w.fp8 else "mla_decode_kernel",
                  "kernel_ms": round(attn_ms, 5)})
     line = {

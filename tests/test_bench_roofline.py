@@ -40,3 +40,19 @@ def test_bound_flips_where_the_roofline_times_cross():
     f_cross = 1e9 / (HBM * 1e9) * TC_BURST * 1e12
     assert bench.attention_roofline(10 ** 9, int(f_cross * 0.99), 1.0, HBM, TC_BURST, TC_SUS)["bound"] == "hbm"
     assert bench.attention_roofline(10 ** 9, int(f_cross * 1.01), 1.0, HBM, TC_BURST, TC_SUS)["bound"] == "tensor"
+
+
+def test_traffic_figures_belong_to_the_current_kernels():
+    # the captured traffic figures are tied to the sources they were captured
+    # with: after a kernel change, capture again (and record the new digest)
+    # or set the entries to None
+    for kernel, digest in bench.ATTN_TRAFFIC_SOURCE_SHA256.items():
+        assert bench.kernel_sources_sha256(kernel) == digest, kernel
+    assert bench.attn_traffic("C2", "mla_decode_kernel") == bench.ATTN_TRAFFIC_BYTES["C2"]
+    assert bench.attn_traffic("C5", "mla_decode_fp8_kernel") == bench.ATTN_TRAFFIC_BYTES["C5"]
+
+
+def test_stale_traffic_is_reported_as_null(monkeypatch):
+    monkeypatch.setitem(bench.ATTN_TRAFFIC_SOURCE_SHA256, "mla_decode_kernel", "0" * 64)
+    assert bench.attn_traffic("C2", "mla_decode_kernel") is None
+    assert bench.attn_traffic("C5", "mla_decode_fp8_kernel") == bench.ATTN_TRAFFIC_BYTES["C5"]
