@@ -37,6 +37,15 @@ catch it:
 - "lo_before_pv": the first part's release is committed before the first PV
   slice is issued.
 
+`abort_at=(t, i)` makes the TMA warp give up at its wait for part i of page
+t, as on a timeout: the other roles stop at once, the copies and MMAs already
+issued complete, and the load lane's drain waits on kv_full for the last page
+it issued into each stage.  Giving up between a page's parts, it first makes
+the page's remaining arrivals.  The drain must end, and end with no copy in
+flight.  Planted mistakes: "no_abort_arrive" (the remaining arrivals are not
+made: the drain never ends) and "extra_abort_arrive" (one arrival too many:
+the drain ends while a part is still landing).
+
 `Fp8Model` (at the end) does the same for the FP8 kernel in
 `csrc/decode_fp8_sm100.cu`, whose protocol differs (three stages filled by 8
 gather warps, QK^T in five parts through a ring of three TMEM slots, V'
@@ -108,8 +117,10 @@ class State:
 
 
 class Model:
-    def __init__(self, plan: Plan, seed: int, mutation: Optional[str] = None, parts: int = REFILL_PARTS):
+    def __init__(self, plan: Plan, seed: int, mutation: Optional[str] = None, parts: int = REFILL_PARTS,
+                 abort_at: Optional[tuple] = None):
         self.plan, self.rng, self.mut, self.parts = plan, random.Random(seed), mutation, parts
+        self.abort_at, self.aborted = abort_at, False
         self.T = sum(plan.segments)
         self.seg_of, self.first_of_seg = [], set()
         t = 0
@@ -135,6 +146,7 @@ class Model:
         self.st.pv_part_done = {i: set() for i in range(parts - 1)}
         self.pipe: List[tuple] = []                  # tensor pipe, in order
         self.loads: List[tuple] = []                 # (page, part) in flight; part 0: chunks 0-3
+        self.last_issued: List[Optional[int]] = [None] * S   # per stage, for the drain after giving up
 
     # -- phase bookkeeping ---------------------------------------------------
     def p_full_phase(self, t):
@@ -150,9 +162,17 @@ class Model:
                     freed = self.kv_empty_part[i - 1]
                 else:
                     freed = self.kv_empty if last else self.kv_empty_part[i]
+                if (t, i) == self.abort_at:
+                    if i > 0 and self.mut != "no_abort_arrive":
+                        for _ in range(self.parts - i + (1 if self.mut == "extra_abort_arrive" else 0)):
+                            self.kv_full[s].arrive(t // STAGES)
+                    self.aborted = True
+                    return
                 yield ("wait", lambda s=s, t=t, freed=freed: freed[s].passes(t // STAGES - 1))
                 self._stage_write_begin(s, t, i)
                 self.loads.append((t, i))
+                if i == 0:
+                    self.last_issued[s] = t
                 yield ("step",)
 
     def mma(self):
@@ -300,6 +320,28 @@ class Model:
             else:
                 self.st.pv_done.add(t)
 
+    def _drain(self):
+        """After the TMA warp gave up: the other roles have stopped; issued
+        copies land and issued MMAs complete in any interleaving until the
+        load lane's waits (kv_full of the last page issued into each stage)
+        all pass."""
+        def drained():
+            return all(lt is None or self.kv_full[s].passes(lt // STAGES) for s, lt in enumerate(self.last_issued))
+        while True:
+            if drained():
+                if self.loads:
+                    raise ProtocolError(f"the drain ends with copies {self.loads} in flight")
+                return
+            movers = [("land", x) for x in self.loads] + ([("pipe", None)] if self.pipe else [])
+            if not movers:
+                raise ProtocolError("the drain never ends: an issued page's kv_full cannot complete")
+            kind, arg = self.rng.choice(movers)
+            if kind == "pipe":
+                self._pipe_pop()
+            else:
+                self.loads.remove(arg)
+                self._land(*arg)
+
     # -- scheduler -------------------------------------------------------------
     def run(self, max_steps: int = 200000):
         roles = [self.mma()] + [self.softmax(w) for w in range(WARPS)] + [self.producer()]
@@ -317,6 +359,9 @@ class Model:
         for i in range(len(roles)):
             advance(i)
         for _ in range(max_steps):
+            if self.aborted:
+                self._drain()
+                return
             if all(done) and not self.pipe and not self.loads:
                 return
             movers, polls = [], []

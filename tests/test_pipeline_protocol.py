@@ -9,7 +9,8 @@ ring of three TMEM slots and the V' rewrite by the gather warps):
 - four softmax warps, with padding warps, lazy rescales, segment epilogues and
   query-tile staging.
 It interleaves them at random, checking parity aliasing, arrivals into the
-wrong phase, data hazards on stages, S, P, Q and O, and deadlock.  The
+wrong phase, data hazards on stages, S, P, Q and O, and deadlock; for the bf16
+kernel also the drain of a CTA whose TMA warp gives up.  The
 current protocol must run clean on every schedule tried.  Each planted
 mistake must be caught."""
 import random
@@ -59,6 +60,29 @@ def test_fp8_planted_mistakes_are_caught(mutation):
         except PM.ProtocolError:
             caught += 1
     assert caught > 0
+
+
+def test_giving_up_drains_every_issued_copy():
+    # the TMA warp gives up at a random wait (between a page's parts too);
+    # the drain at exit must end, and end with nothing in flight
+    for parts in (2, 4):
+        for seed in range(200):
+            rng = random.Random(seed)
+            plan = _plan(rng, False)
+            PM.Model(plan, seed, parts=parts, abort_at=(rng.randrange(sum(plan.segments)), rng.randrange(parts))).run()
+
+
+@pytest.mark.parametrize("mutation", ["no_abort_arrive", "extra_abort_arrive"])
+def test_planted_drain_mistakes_are_caught(mutation):
+    caught = 0
+    for seed in range(40):
+        rng = random.Random(seed)
+        plan = _plan(rng, False)
+        try:
+            PM.Model(plan, seed, mutation=mutation, abort_at=(rng.randrange(sum(plan.segments)), 1)).run()
+        except PM.ProtocolError:
+            caught += 1
+    assert caught == 40
 
 
 @pytest.mark.parametrize("mutation", ["shared_p_full", "no_rescale_wait", "single_pv_barrier", "hi_on_lo",
