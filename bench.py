@@ -62,7 +62,7 @@ ATTN_KERNEL_SOURCES = {
                               "mla_api.cu"),
 }
 ATTN_TRAFFIC_SOURCE_SHA256 = {
-    "mla_decode_kernel": "981accf908896c80338a1b3917dcf53f4876aa1d9f0032097acae137c2649c45",
+    "mla_decode_kernel": "6ed14556c1d04e02372428e056698d7e51bdd43ea699c8e8c43a2f2f6d5c1385",
     "mla_decode_fp8_kernel": "f1eec4739e0e4722b0ffc0743a1864e3251956a1efe280d46b9c9cdf967d7c52",
 }
 

@@ -159,8 +159,9 @@ static_assert(kStages == 3, "Issued holds three stages");
 // Warp 0 (one lane): TMA loads of cache pages, each in two parts (chunks 0-3
 // once the stage's first PV half has completed, chunks 4-8 once all of PV
 // has), their block-table entries read kPrefetchPages pages ahead, and an L2
-// prefetch of the next segment's query tile.  (Warming the pages themselves in L2 ahead of their loads, 1 to
-// 4 pages ahead, measured slower than not warming them at all.)
+// prefetch of the next segment's query tile.  (Warming the pages themselves
+// in L2 ahead of their loads, 1 to 4 pages ahead, measured slower than not
+// warming them at all.)
 __device__ __forceinline__ void load_role(const DecodeParams& p, const Partition& part, const CUtensorMap* tmap_kv,
                                           uint8_t* smem, Bars bars, StageInfo* info, volatile int* abort_flag,
                                           Issued& issued) {
