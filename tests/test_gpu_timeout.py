@@ -29,6 +29,9 @@ def _workload(case):
     return I.make_workload("tofp8s", 2, 1, 64, [3000, 1000], fp8=True, topk=1024, seed=83)
 
 
+# the outputs of the call that gave up are undefined (numpy warns on casting
+# their garbage); only its error word is checked
+@pytest.mark.filterwarnings("ignore:invalid value encountered in cast:RuntimeWarning")
 @pytest.mark.parametrize("case", ["bf16", "fp8 dense", "fp8 sparse"])
 def test_waits_give_up_and_the_next_call_is_correct(case):
     w = _workload(case)
